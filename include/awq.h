@@ -1,0 +1,147 @@
+/*
+ * awq.h -- C ABI of the B200 (sm_100a) AWQ hot-path library (libawq_b200.so).
+ *
+ * AWQ, activation-aware weight quantization (MIT Han Lab; described on the robotsatlas.com
+ * "AWQ" page, sections "How it works", "Key mechanisms", "Components" and
+ * "Hyperparameters", and on the builderai.tools "AWQ" page, section "About"):
+ *   1. measure each input channel's activation magnitude on a calibration set,
+ *   2. scale salient weight channels up by s (and the activations down by s),
+ *   3. pick s on a grid by minimising the layer's output error,
+ *   4. quantize the scaled weights group-wise to 4 (or 3) bits with a per-group scale,
+ *   5. run the layer with kernels that take the packed weights and fp16 activations.
+ *
+ * Conventions shared by every call
+ *   - Tensors are row-major. W is [N, K] (N output features, K input channels); X is
+ *     [M, K] (M tokens); Y = X W^T is [M, N]. fp16 means IEEE binary16 (awq_f16 below).
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller and must be 16-byte
+ *     aligned. The library never allocates device memory: calls that need scratch space
+ *     take a caller-owned workspace whose size the matching *_workspace_size query gives.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Every
+ *     call is asynchronous on it; outputs are valid once the stream reaches that point.
+ *   - The group size must be 128 and K a multiple of 128; bits is 4 or 3.
+ *   - Dimensions must be below 2^31.
+ *   - Arguments are checked on the host before anything is launched: a call that returns
+ *     an error other than AWQ_ERR_CUDA has launched nothing and written nothing.
+ *   - Kernels bound every internal wait (about 2 s); a wait that runs out sets a device
+ *     status word that awq_check_error() reports as AWQ_ERR_TIMEOUT.
+ *   - Calls on one stream are ordered; calls that share a workspace must not overlap.
+ *
+ * Packed weight layout (this library's convention; the pages fix only "group-wise 4-bit
+ * with a per-group scale, e.g. groups of 128"):
+ *   - 4-bit: qweight is uint32 [N, K/8]; word j of row n holds k = 8j..8j+7, the code of
+ *     k-offset i in nibble position i/2 + 4*(i%2) (positions 0..7 hold offsets
+ *     0,2,4,6,1,3,5,7), so masks 0x000F000F / 0x00F000F0 on the word and on the word
+ *     shifted right by 8 yield the consecutive pairs (k0,k1), (k2,k3), (k4,k5), (k6,k7).
+ *   - 3-bit: qweight is uint32 [N, 3K/32]; per block of 32 consecutive k, word 0 holds the
+ *     low two bits of offsets 0..15 and word 1 those of 16..31 (offset i mod 16 at 2-bit
+ *     field i/2 + 8*(i%2)), word 2 holds bit 2 of offset i at bit i/2 + 16*(i%2).
+ *   - scales: fp16 [K/128, N]; zeros: uint8 [K/128, N] (group-major).
+ *   - Dequantized weight: (q - zero) * scale. Storage: 4.1875 bits per weight at 4 bits,
+ *     3.1875 at 3 bits.
+ */
+#ifndef AWQ_B200_H_
+#define AWQ_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AWQ_API __attribute__((visibility("default")))
+#else
+#define AWQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t awq_f16; /* IEEE binary16 storage */
+
+typedef enum {
+  AWQ_OK = 0,
+  AWQ_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad shape, unsupported bits/group */
+  AWQ_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement */
+  AWQ_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the size query's answer */
+  AWQ_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (e.g. no GPU, launch) */
+  AWQ_ERR_TIMEOUT = 5        /* a kernel's bounded wait ran out (see awq_check_error) */
+} awq_status;
+
+/* Human-readable name of a status code. Never NULL. */
+AWQ_API const char* awq_status_string(awq_status status);
+
+/* Version of this ABI (bumped on any signature or layout change). */
+AWQ_API int awq_abi_version(void);
+
+/* Synchronises `stream`, then reads and clears the device status word of the current
+ * device. Returns AWQ_ERR_TIMEOUT if a kernel reported a bounded-wait timeout since the
+ * last check, AWQ_ERR_CUDA if the synchronisation failed, AWQ_OK otherwise. */
+AWQ_API awq_status awq_check_error(void* stream);
+
+/* ---------------------------------------------------------------- activation statistics
+ * robotsatlas.com "AWQ", "How it works" / "Components: Activation saliency analysis":
+ * the activation magnitude of every input channel on the calibration set,
+ *     s_x[k] = (1/M) * sum_m |X[m, k]|      (fp64 accumulation, rounded once to fp32).
+ * X: fp16 [M, K], M >= 1, K a multiple of 8. s_x: fp32 [K] (output).
+ * workspace: at least awq_act_stats_workspace_size(M, K) bytes (fp64 partial sums). */
+AWQ_API size_t awq_act_stats_workspace_size(int64_t M, int64_t K);
+AWQ_API awq_status awq_act_stats(const awq_f16* X, int64_t M, int64_t K, float* s_x, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- quantize and pack
+ * robotsatlas.com "AWQ", "Components: Group-wise 4-bit quantization" and "Hyperparameters";
+ * builderai.tools "AWQ", "About" ("writes real INT4 weights"). Quantizes W diag(s) per
+ * (row, group of 128) with an asymmetric code, in IEEE fp32 with one rounding per step:
+ *     w' = w * s[k]; scale = max((max w' - min w') / qmax, 1e-5) rounded to fp16 (sc);
+ *     z = clamp(rint(-min w' / sc), 0, qmax); q = clamp(rint(w' / sc) + z, 0, qmax),
+ * qmax = 2^bits - 1, rint = round half to even.
+ * W: fp16 [N, K]. s: fp32 [K], or NULL for s = 1 (plain round-to-nearest).
+ * Outputs: qweight (layout above), scales fp16 [K/128, N], zeros uint8 [K/128, N].
+ * N = 0 is a no-op. K % 128 == 0 (and K % 32 == 0 for 3 bits). No workspace. */
+AWQ_API awq_status awq_quantize_pack(const awq_f16* W, int64_t N, int64_t K, const float* s, int bits,
+                             int group, uint32_t* qweight, awq_f16* scales, uint8_t* zeros,
+                             void* stream);
+
+/* ---------------------------------------------------------------- scale search
+ * robotsatlas.com "AWQ", "How it works" and "Key mechanisms": per-channel scale chosen by a
+ * grid search that minimises the layer's output error. For every grid point a,
+ *     s_a[k]  = max(s_x[k], 1e-4)^alphas[a]            (fp64 pow, rounded to fp32), or
+ *               s_table[a][k] when s_table is not NULL,
+ *     L[a]    = || (deq(Q(W diag(s_a))) diag(1/s_a)) X^T - W X^T ||_F^2,
+ * with Q the quantizer of awq_quantize_pack. The error operand
+ * E_a = fp16(deq * (1/s_a) - W) is formed per grid point and L[a] = ||E_a X^T||^2 is
+ * evaluated on the tensor cores (fp16 operands, fp32 accumulation, fp64 reduction in a
+ * fixed order). best_idx = the first index of the minimum; best_s = s_{best_idx}.
+ * Searching q/k/v (or gate/up) jointly = passing their row-concatenated W.
+ * W: fp16 [N, K]; X: fp16 [M, K] (calibration tokens); s_x: fp32 [K]; alphas: fp32 device
+ * array [n_alpha] (1 <= n_alpha <= 64); s_table: NULL or fp32 [n_alpha, K].
+ * Outputs (device): losses fp64 [n_alpha], best_idx int32 [1], best_s fp32 [K],
+ * row_losses NULL or fp64 [n_alpha, N] (each row's share of L[a]).
+ * workspace: at least awq_search_scale_workspace_size(M, N, K, n_alpha) bytes. */
+AWQ_API size_t awq_search_scale_workspace_size(int64_t M, int64_t N, int64_t K, int n_alpha);
+AWQ_API awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f16* X,
+                            int64_t M, const float* s_x, const float* alphas, int n_alpha,
+                            int bits, int group, const float* s_table, double* losses,
+                            int32_t* best_idx, float* best_s, double* row_losses,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- W4A16 GEMM
+ * builderai.tools "AWQ", "About" (kernels for 4-bit weights with 16-bit activations);
+ * robotsatlas.com "AWQ", "Implementation pitfalls" (dequantization fused into the GEMM).
+ *     Y[m, n] = sum_k x'[m, k] * (q[n, k] - z[k/128, n]) * scale[k/128, n]
+ * with x' = X, or x' = fp16(X[m, k] * inv_s[k]) when inv_s is not NULL (the activation side
+ * of the per-channel scaling). fp32 accumulation, fp16 output.
+ * M <= 16 with 4 bits runs the decode kernel (HBM-bound GEMV); larger M (and 3 bits) the
+ * tensor-core kernel. X: fp16 [M, K]; Y: fp16 [M, N]. M = 0 or N = 0 is a no-op.
+ * workspace: at least awq_gemm_workspace_size(M, N, K, bits) bytes (0 when inv_s is NULL
+ * or M <= 16). */
+AWQ_API size_t awq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits);
+AWQ_API awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
+                          const awq_f16* scales, const uint8_t* zeros, int64_t N, int64_t K,
+                          int bits, int group, const float* inv_s, awq_f16* Y, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AWQ_B200_H_ */

@@ -1,0 +1,95 @@
+"""The C-ABI library builds, loads without a GPU, exports every entry point that include/*.h
+declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _lib():
+    from weight_only_int4_stats_b200 import build
+    build.build()
+    import weight_only_int4_stats_b200 as awq
+    return awq.lib()
+
+
+def _declared():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names += re.findall(r"^AWQ_API\s+[\w\s\*]+?\b(awq_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = set(_declared())
+    for want in ("awq_act_stats", "awq_search_scale", "awq_quantize_pack", "awq_gemm_w4a16",
+                 "awq_act_stats_workspace_size", "awq_search_scale_workspace_size",
+                 "awq_gemm_workspace_size", "awq_check_error", "awq_status_string",
+                 "awq_abi_version"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = _lib()
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings_and_version():
+    L = _lib()
+    for code, name in enumerate(["AWQ_OK", "AWQ_ERR_INVALID_ARG", "AWQ_ERR_UNSUPPORTED",
+                                 "AWQ_ERR_WORKSPACE", "AWQ_ERR_CUDA", "AWQ_ERR_TIMEOUT"]):
+        assert L.awq_status_string(code).decode() == name
+    assert L.awq_abi_version() == 1
+
+
+def test_host_validation_rejects_before_launch():
+    L = _lib()
+    P = ctypes.c_void_p
+    fake = P(1 << 20)          # never dereferenced: every call below fails validation first
+    odd = P((1 << 20) + 2)     # misaligned
+    # act_stats: null X, M = 0, K not a multiple of 8
+    assert L.awq_act_stats(None, 4, 8, fake, fake, 1 << 20, None) == 1
+    assert L.awq_act_stats(fake, 0, 8, fake, fake, 1 << 20, None) == 1
+    assert L.awq_act_stats(fake, 4, 12, fake, fake, 1 << 20, None) == 1
+    assert L.awq_act_stats(odd, 4, 8, fake, fake, 1 << 20, None) == 1
+    # quantize_pack: bad bits, bad group, K not a multiple of 128; N = 0 is a no-op
+    assert L.awq_quantize_pack(fake, 4, 128, None, 5, 128, fake, fake, fake, None) == 1
+    assert L.awq_quantize_pack(fake, 4, 128, None, 4, 64, fake, fake, fake, None) == 1
+    assert L.awq_quantize_pack(fake, 4, 200, None, 4, 128, fake, fake, fake, None) == 1
+    assert L.awq_quantize_pack(fake, 0, 128, None, 4, 128, fake, fake, fake, None) == 0
+    # gemm: M = 0 and N = 0 are no-ops; misaligned Y; bits 2
+    assert L.awq_gemm_w4a16(fake, 0, fake, fake, fake, 8, 128, 4, 128, None, fake, None, 0,
+                            None) == 0
+    assert L.awq_gemm_w4a16(fake, 1, fake, fake, fake, 0, 128, 4, 128, None, fake, None, 0,
+                            None) == 0
+    assert L.awq_gemm_w4a16(fake, 1, fake, fake, fake, 8, 128, 4, 128, None, odd, None, 0,
+                            None) == 1
+    assert L.awq_gemm_w4a16(fake, 1, fake, fake, fake, 8, 128, 2, 128, None, fake, None, 0,
+                            None) == 1
+    # search: n_alpha out of range, too-small workspace
+    assert L.awq_search_scale(fake, 8, 128, fake, 4, fake, fake, 0, 4, 128, None, fake, fake,
+                              fake, None, fake, 1 << 30, None) == 1
+    assert L.awq_search_scale(fake, 8, 128, fake, 4, fake, fake, 20, 4, 128, None, fake, fake,
+                              fake, None, fake, 16, None) == 3
+
+
+def test_workspace_queries():
+    L = _lib()
+    assert L.awq_search_scale_workspace_size(256, 512, 512, 20) >= 20 * 512 * 512 * 2
+    assert L.awq_gemm_workspace_size(1, 4096, 4096, 4) == 0
+    assert L.awq_gemm_workspace_size(2048, 4096, 4096, 4) >= 2048 * 4096 * 2
+    assert L.awq_act_stats_workspace_size(0, 16) == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import weight_only_int4_stats_b200 as awq
+    monkeypatch.setattr(awq, "library_path", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(awq, "_lib", None)
+    with pytest.raises(ImportError):
+        awq.lib()

@@ -1,0 +1,184 @@
+"""AWQ hot path on B200: a thin Python binding over libawq_b200.so (include/awq.h).
+
+Every function here only marshals arguments: it checks dtypes, allocates outputs and the
+workspace with PyTorch (device memory and the current stream are PyTorch's), and calls the
+C entry point of the same name. All arithmetic runs in the library's CUDA kernels. There is
+no fallback: if the library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "AwqError", "lib", "library_path", "GROUP",
+    "awq_act_stats", "awq_quantize_pack", "awq_search_scale", "awq_gemm_w4a16",
+    "awq_check_error", "packed_words_per_row",
+]
+
+GROUP = 128
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libawq_b200.so")
+
+STATUS = {0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_UNSUPPORTED",
+          3: "AWQ_ERR_WORKSPACE", 4: "AWQ_ERR_CUDA", 5: "AWQ_ERR_TIMEOUT"}
+
+
+class AwqError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+        self.status = STATUS.get(code, str(code))
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library (loaded on first use; raises if it was never built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise ImportError(
+                f"{library_path} is missing: build it with "
+                "`python -m weight_only_int4_stats_b200.build` (there is no CPU fallback)")
+        L = ctypes.CDLL(library_path)
+        P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        sig = {
+            "awq_status_string": (ctypes.c_char_p, [I32]),
+            "awq_abi_version": (I32, []),
+            "awq_check_error": (I32, [P]),
+            "awq_act_stats_workspace_size": (SZ, [I64, I64]),
+            "awq_act_stats": (I32, [P, I64, I64, P, P, SZ, P]),
+            "awq_quantize_pack": (I32, [P, I64, I64, P, I32, I32, P, P, P, P]),
+            "awq_search_scale_workspace_size": (SZ, [I64, I64, I64, I32]),
+            "awq_search_scale": (I32, [P, I64, I64, P, I64, P, P, I32, I32, I32, P, P, P, P, P,
+                                       P, SZ, P]),
+            "awq_gemm_workspace_size": (SZ, [I64, I64, I64, I32]),
+            "awq_gemm_w4a16": (I32, [P, I64, P, P, P, I64, I64, I32, I32, P, P, P, SZ, P]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise AwqError(fn, code)
+
+
+def _need(t, dtype, name):
+    if t is None:
+        return
+    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name}: expected a contiguous CUDA tensor of {dtype}, got "
+                        f"{t.dtype} on {t.device} (contiguous={t.is_contiguous()})")
+
+
+def _workspace(nbytes: int, device):
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def packed_words_per_row(K: int, bits: int) -> int:
+    return K // 8 if bits == 4 else 3 * K // 32
+
+
+def awq_check_error(stream=None) -> None:
+    _check("awq_check_error", lib().awq_check_error(_stream(stream)))
+
+
+def awq_act_stats(X: torch.Tensor, out: torch.Tensor | None = None, workspace=None,
+                  stream=None) -> torch.Tensor:
+    """s_x[k] = mean_m |X[m, k]| (fp32 [K]) for fp16 X [M, K]."""
+    _need(X, torch.float16, "X")
+    M, K = X.shape
+    s_x = torch.empty(K, dtype=torch.float32, device=X.device) if out is None else out
+    _need(s_x, torch.float32, "out")
+    ws_bytes = lib().awq_act_stats_workspace_size(M, K)
+    ws = _workspace(ws_bytes, X.device) if workspace is None else workspace
+    _check("awq_act_stats", lib().awq_act_stats(_ptr(X), M, K, _ptr(s_x), _ptr(ws),
+                                                ws.numel() * ws.element_size(), _stream(stream)))
+    return s_x
+
+
+def awq_quantize_pack(W: torch.Tensor, s: torch.Tensor | None, bits: int = 4,
+                      group: int = GROUP, out=None, stream=None):
+    """Quantize W diag(s) group-wise and pack: (qweight uint32 as int32, scales fp16 [G, N],
+    zeros uint8 [G, N])."""
+    _need(W, torch.float16, "W")
+    _need(s, torch.float32, "s")
+    N, K = W.shape
+    dev = W.device
+    if out is None:
+        qweight = torch.empty(N, packed_words_per_row(K, bits), dtype=torch.int32, device=dev)
+        scales = torch.empty(K // group, N, dtype=torch.float16, device=dev)
+        zeros = torch.empty(K // group, N, dtype=torch.uint8, device=dev)
+    else:
+        qweight, scales, zeros = out
+    _check("awq_quantize_pack", lib().awq_quantize_pack(
+        _ptr(W), N, K, _ptr(s), bits, group, _ptr(qweight), _ptr(scales), _ptr(zeros),
+        _stream(stream)))
+    return qweight, scales, zeros
+
+
+def awq_search_scale(W: torch.Tensor, X: torch.Tensor, s_x: torch.Tensor | None,
+                     alphas: torch.Tensor | None, bits: int = 4, group: int = GROUP,
+                     s_table: torch.Tensor | None = None, row_losses: bool = False,
+                     workspace=None, stream=None):
+    """Grid search of the per-channel scale. Returns (losses fp64 [A], best_idx int32 [1],
+    best_s fp32 [K], row_losses fp64 [A, N] or None)."""
+    _need(W, torch.float16, "W")
+    _need(X, torch.float16, "X")
+    _need(s_x, torch.float32, "s_x")
+    _need(alphas, torch.float32, "alphas")
+    _need(s_table, torch.float32, "s_table")
+    N, K = W.shape
+    M = X.shape[0]
+    A = alphas.numel() if alphas is not None else s_table.shape[0]
+    dev = W.device
+    losses = torch.empty(A, dtype=torch.float64, device=dev)
+    best_idx = torch.empty(4, dtype=torch.int32, device=dev)
+    best_s = torch.empty(K, dtype=torch.float32, device=dev)
+    rl = torch.empty(A, N, dtype=torch.float64, device=dev) if row_losses else None
+    ws_bytes = lib().awq_search_scale_workspace_size(M, N, K, A)
+    ws = _workspace(ws_bytes, dev) if workspace is None else workspace
+    _check("awq_search_scale", lib().awq_search_scale(
+        _ptr(W), N, K, _ptr(X), M, _ptr(s_x), _ptr(alphas), A, bits, group, _ptr(s_table),
+        _ptr(losses), _ptr(best_idx), _ptr(best_s), _ptr(rl), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    return losses, best_idx[:1], best_s, rl
+
+
+def awq_gemm_w4a16(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+                   zeros: torch.Tensor, N: int, K: int, bits: int = 4, group: int = GROUP,
+                   inv_s: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                   workspace=None, stream=None) -> torch.Tensor:
+    """Y = X deq(W)^T (fp16 [M, N]) with the dequantization fused into the kernel."""
+    _need(X, torch.float16, "X")
+    _need(scales, torch.float16, "scales")
+    _need(zeros, torch.uint8, "zeros")
+    _need(inv_s, torch.float32, "inv_s")
+    M = X.shape[0]
+    Y = torch.empty(M, N, dtype=torch.float16, device=X.device) if out is None else out
+    ws = workspace
+    if ws is None and inv_s is not None:
+        ws = _workspace(lib().awq_gemm_workspace_size(M, N, K, bits), X.device)
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("awq_gemm_w4a16", lib().awq_gemm_w4a16(
+        _ptr(X), M, _ptr(qweight), _ptr(scales), _ptr(zeros), N, K, bits, group, _ptr(inv_s),
+        _ptr(Y), _ptr(ws), ws_bytes, _stream(stream)))
+    return Y

@@ -1,0 +1,61 @@
+"""Builds libawq_b200.so in place (sm_100a only).
+
+    python -m weight_only_int4_stats_b200.build [--verbose-ptxas]
+
+nvcc cross-compiles without a GPU. The CUDA runtime is linked statically and the driver's
+tensor-map encoder is looked up at run time, so the library loads on a machine without a
+GPU (every call then returns AWQ_ERR_CUDA).
+"""
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+LIB = os.path.join(PKG, "libawq_b200.so")
+SOURCES = [os.path.join(PKG, "csrc", "awq_api.cu")]
+DEPS = [os.path.join(PKG, "csrc", f) for f in os.listdir(os.path.join(PKG, "csrc"))] + [
+    os.path.join(ROOT, "include", "awq.h")]
+
+
+def nvcc_path() -> str:
+    p = shutil.which("nvcc")
+    if p:
+        return p
+    p = "/usr/local/cuda/bin/nvcc"
+    if os.path.exists(p):
+        return p
+    raise RuntimeError("nvcc not found")
+
+
+def command(verbose_ptxas: bool = False) -> list[str]:
+    cmd = [
+        nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
+        "-std=c++17", "-shared", "-Xcompiler", "-fPIC,-fvisibility=hidden",
+        "-I", os.path.join(ROOT, "include"), "-I", os.path.join(PKG, "csrc"),
+        "-o", LIB,
+    ] + SOURCES
+    if verbose_ptxas:
+        cmd[1:1] = ["-Xptxas", "-v"]
+    return cmd
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    t = os.path.getmtime(LIB)
+    return all(os.path.getmtime(d) <= t for d in DEPS if os.path.exists(d))
+
+
+def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+    if force or verbose_ptxas or not up_to_date():
+        subprocess.run(command(verbose_ptxas), check=True)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv)
+    print(LIB)

@@ -1,0 +1,366 @@
+// Host side of the C ABI declared in include/awq.h: argument checks, workspace carving,
+// TMA descriptor encoding and kernel dispatch. All kernels live in the *.cuh files of this
+// directory and are compiled into this one translation unit for sm_100a.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "awq.h"
+#include "act_stats.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "quantize.cuh"
+#include "search.cuh"
+
+namespace {
+
+using awq::ASrc;
+using awq::Epi;
+
+constexpr int64_t kMaxDim = (int64_t{1} << 31) - 1;
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+size_t align256(size_t v) { return (v + 255) & ~size_t{255}; }
+
+awq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA; }
+
+awq_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+int num_sms() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `elem` bytes per element; box [box_rows, box_cols].
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem,
+                  int64_t rows, int64_t cols, int box_rows, int box_cols, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * elem};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, ASrc kA, Epi kEpi>
+awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_rows,
+                     const awq::TcArgs& args, cudaStream_t st) {
+  using L = awq::TcLayout<BN, kA>;
+  static bool attr_set[kMaxDevices] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
+  auto kern = awq::tc_gemm_kernel<BN, kA, kEpi>;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem) !=
+        cudaSuccess)
+      return AWQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tx, ta;
+  if (!make_tmap_2d(&tx, Xop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, args.K, BN, awq::kTcBK,
+                    true))
+    return AWQ_ERR_CUDA;
+  if (kA == ASrc::kFp16) {
+    if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a_rows, args.K, awq::kTcBM,
+                      awq::kTcBK, true))
+      return AWQ_ERR_CUDA;
+  } else {
+    if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a_rows, args.K / 8,
+                      awq::kTcBM, awq::kTcBK / 8, false))
+      return AWQ_ERR_CUDA;
+  }
+  dim3 grid(static_cast<unsigned>((M + BN - 1) / BN),
+            static_cast<unsigned>((a_rows + awq::kTcBM - 1) / awq::kTcBM));
+  kern<<<grid, awq::kTcThreads, L::kSmem, st>>>(tx, ta, args);
+  return launch_status();
+}
+
+template <ASrc kA, Epi kEpi>
+awq_status launch_tc_bn(const __half* Xop, int64_t M, const void* Aop, int64_t a_rows,
+                        const awq::TcArgs& args, cudaStream_t st) {
+  if (M <= 32) return launch_tc<32, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
+  if (M <= 64) return launch_tc<64, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
+  if (M <= 128) return launch_tc<128, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
+  return launch_tc<256, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
+}
+
+int tc_bn_for(int64_t M) { return M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
+
+bool bad_dim(int64_t v) { return v < 0 || v > kMaxDim; }
+
+}  // namespace
+
+extern "C" {
+
+const char* awq_status_string(awq_status status) {
+  switch (status) {
+    case AWQ_OK: return "AWQ_OK";
+    case AWQ_ERR_INVALID_ARG: return "AWQ_ERR_INVALID_ARG";
+    case AWQ_ERR_UNSUPPORTED: return "AWQ_ERR_UNSUPPORTED";
+    case AWQ_ERR_WORKSPACE: return "AWQ_ERR_WORKSPACE";
+    case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA";
+    case AWQ_ERR_TIMEOUT: return "AWQ_ERR_TIMEOUT";
+  }
+  return "AWQ_ERR_UNKNOWN";
+}
+
+int awq_abi_version(void) { return 1; }
+
+awq_status awq_check_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return AWQ_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, awq::g_status_word, sizeof(word)) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(awq::g_status_word, &zero, sizeof(zero)) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  if (word & awq::kDevErrTimeout) return AWQ_ERR_TIMEOUT;
+  return AWQ_OK;
+}
+
+// ------------------------------------------------------------------ act_stats
+size_t awq_act_stats_workspace_size(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0) return 0;
+  const int splits = awq::act_stats_splits(M, K, num_sms());
+  return static_cast<size_t>(splits) * static_cast<size_t>(K) * sizeof(double);
+}
+
+awq_status awq_act_stats(const awq_f16* X, int64_t M, int64_t K, float* s_x, void* workspace,
+                         size_t ws_bytes, void* stream) {
+  if (bad_dim(M) || bad_dim(K) || M == 0) return AWQ_ERR_INVALID_ARG;
+  if (K == 0) return AWQ_OK;
+  if (K % 8 != 0) return AWQ_ERR_INVALID_ARG;
+  if (!X || !s_x || !aligned16(X) || !aligned16(s_x)) return AWQ_ERR_INVALID_ARG;
+  const int splits = awq::act_stats_splits(M, K, num_sms());
+  const size_t need = static_cast<size_t>(splits) * static_cast<size_t>(K) * sizeof(double);
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return AWQ_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  double* part = static_cast<double*>(workspace);
+  const int64_t rows_per_split = (M + splits - 1) / splits;
+  dim3 g1(static_cast<unsigned>((K + awq::kStatsCols - 1) / awq::kStatsCols),
+          static_cast<unsigned>(splits));
+  awq::act_stats_partial_kernel<<<g1, 256, 0, st>>>(reinterpret_cast<const __half*>(X), M, K,
+                                                   rows_per_split, part);
+  awq_status s = launch_status();
+  if (s != AWQ_OK) return s;
+  awq::act_stats_finish_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(
+      part, splits, M, K, s_x);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ quantize_pack
+awq_status awq_quantize_pack(const awq_f16* W, int64_t N, int64_t K, const float* s, int bits,
+                             int group, uint32_t* qweight, awq_f16* scales, uint8_t* zeros,
+                             void* stream) {
+  if (bad_dim(N) || bad_dim(K) || K == 0) return AWQ_ERR_INVALID_ARG;
+  if (group != awq::kGroup || K % awq::kGroup != 0) return AWQ_ERR_INVALID_ARG;
+  if (bits != 4 && bits != 3) return AWQ_ERR_INVALID_ARG;
+  if (N == 0) return AWQ_OK;
+  if (!W || !qweight || !scales || !zeros) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
+      (s && !aligned16(s)))
+    return AWQ_ERR_INVALID_ARG;
+  if ((K / awq::kGroup) > 65535) return AWQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dim3 grid(static_cast<unsigned>((N + awq::kQuantRowsPerCta - 1) / awq::kQuantRowsPerCta),
+            static_cast<unsigned>(K / awq::kGroup));
+  const __half* w = reinterpret_cast<const __half*>(W);
+  __half* sc = reinterpret_cast<__half*>(scales);
+  if (bits == 4)
+    awq::quantize_pack_kernel<4><<<grid, 256, 0, st>>>(w, N, K, s, qweight, sc, zeros);
+  else
+    awq::quantize_pack_kernel<3><<<grid, 256, 0, st>>>(w, N, K, s, qweight, sc, zeros);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ search
+namespace {
+struct SearchWs {
+  size_t table, err, part, total;
+};
+SearchWs search_ws_layout(int64_t M, int64_t N, int64_t K, int n_alpha) {
+  const int64_t N_pad = round_up(N, awq::kTcBM);
+  const int64_t m_tiles = (M + tc_bn_for(M) - 1) / tc_bn_for(M);
+  SearchWs w;
+  w.table = 0;
+  w.err = align256(static_cast<size_t>(n_alpha) * K * sizeof(float));
+  w.part = w.err + align256(static_cast<size_t>(n_alpha) * N_pad * K * sizeof(__half));
+  w.total = w.part + align256(static_cast<size_t>(n_alpha) * N_pad * m_tiles * sizeof(double));
+  return w;
+}
+}  // namespace
+
+size_t awq_search_scale_workspace_size(int64_t M, int64_t N, int64_t K, int n_alpha) {
+  if (M <= 0 || N <= 0 || K <= 0 || n_alpha <= 0) return 0;
+  return search_ws_layout(M, N, K, n_alpha).total;
+}
+
+awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f16* X,
+                            int64_t M, const float* s_x, const float* alphas, int n_alpha,
+                            int bits, int group, const float* s_table, double* losses,
+                            int32_t* best_idx, float* best_s, double* row_losses,
+                            void* workspace, size_t ws_bytes, void* stream) {
+  if (bad_dim(N) || bad_dim(K) || bad_dim(M) || N == 0 || K == 0 || M == 0)
+    return AWQ_ERR_INVALID_ARG;
+  if (group != awq::kGroup || K % awq::kGroup != 0) return AWQ_ERR_INVALID_ARG;
+  if (bits != 4 && bits != 3) return AWQ_ERR_INVALID_ARG;
+  if (n_alpha < 1 || n_alpha > 64) return AWQ_ERR_INVALID_ARG;
+  if (!W || !X || !losses || !best_idx || !best_s) return AWQ_ERR_INVALID_ARG;
+  if (!s_table && (!s_x || !alphas)) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(X) || !aligned16(losses) || !aligned16(best_idx) ||
+      !aligned16(best_s) || (s_x && !aligned16(s_x)) || (alphas && !aligned16(alphas)) ||
+      (s_table && !aligned16(s_table)) || (row_losses && !aligned16(row_losses)))
+    return AWQ_ERR_INVALID_ARG;
+  const int64_t N_pad = round_up(N, awq::kTcBM);
+  if (n_alpha * N_pad / awq::kTcBM > 65535 || K / awq::kGroup > 65535)
+    return AWQ_ERR_INVALID_ARG;
+  const SearchWs lay = search_ws_layout(M, N, K, n_alpha);
+  if (!workspace || ws_bytes < lay.total || !aligned16(workspace)) return AWQ_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* table = reinterpret_cast<float*>(ws + lay.table);
+  __half* E = reinterpret_cast<__half*>(ws + lay.err);
+  double* part = reinterpret_cast<double*>(ws + lay.part);
+  const int bn = tc_bn_for(M);
+  const int m_tiles = static_cast<int>((M + bn - 1) / bn);
+  awq_status s;
+
+  const float* S = s_table;
+  if (S == nullptr) {
+    dim3 g(static_cast<unsigned>((K + 255) / 256), static_cast<unsigned>(n_alpha));
+    awq::scale_candidates_kernel<<<g, 256, 0, st>>>(s_x, alphas, n_alpha, K, table);
+    if ((s = launch_status()) != AWQ_OK) return s;
+    S = table;
+  }
+  {
+    dim3 g(static_cast<unsigned>(N_pad / awq::kQuantRowsPerCta),
+           static_cast<unsigned>(K / awq::kGroup), static_cast<unsigned>(n_alpha));
+    const __half* w = reinterpret_cast<const __half*>(W);
+    if (bits == 4)
+      awq::search_build_error_kernel<4><<<g, 256, 0, st>>>(w, N, K, N_pad, S, E);
+    else
+      awq::search_build_error_kernel<3><<<g, 256, 0, st>>>(w, N, K, N_pad, S, E);
+    if ((s = launch_status()) != AWQ_OK) return s;
+  }
+  {
+    awq::TcArgs args{};
+    args.M = M;
+    args.N = N;
+    args.N_pad = N_pad;
+    args.K = K;
+    args.row_part = part;
+    args.m_tiles = m_tiles;
+    s = launch_tc_bn<ASrc::kFp16, Epi::kRowSumSq>(reinterpret_cast<const __half*>(X), M, E,
+                                                  n_alpha * N_pad, args, st);
+    if (s != AWQ_OK) return s;
+  }
+  awq::search_reduce_kernel<<<n_alpha, awq::kReduceThreads, 0, st>>>(part, N, N_pad, m_tiles,
+                                                                     row_losses, losses);
+  if ((s = launch_status()) != AWQ_OK) return s;
+  awq::search_pick_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(
+      losses, n_alpha, S, K, best_idx, best_s);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ GEMM
+size_t awq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits) {
+  (void)N;
+  if (M <= 0 || K <= 0) return 0;
+  if (M <= 16 && bits == 4) return 0;
+  return align256(static_cast<size_t>(M) * K * sizeof(__half));
+}
+
+awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
+                          const awq_f16* scales, const uint8_t* zeros, int64_t N, int64_t K,
+                          int bits, int group, const float* inv_s, awq_f16* Y, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  if (bad_dim(M) || bad_dim(N) || bad_dim(K) || K == 0) return AWQ_ERR_INVALID_ARG;
+  if (group != awq::kGroup || K % awq::kGroup != 0) return AWQ_ERR_INVALID_ARG;
+  if (bits != 4 && bits != 3) return AWQ_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return AWQ_OK;
+  if (!X || !qweight || !scales || !zeros || !Y) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
+      !aligned16(Y) || (inv_s && !aligned16(inv_s)))
+    return AWQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const __half* x = reinterpret_cast<const __half*>(X);
+  const __half* sc = reinterpret_cast<const __half*>(scales);
+  __half* y = reinterpret_cast<__half*>(Y);
+
+  if (M <= 16 && bits == 4) {
+    const unsigned grid = static_cast<unsigned>((N + awq::kGemvRows - 1) / awq::kGemvRows);
+    if (M <= 8)
+      awq::gemv_w4a16_kernel<1><<<grid, awq::kGemvWarps * 32, 0, st>>>(
+          x, static_cast<int>(M), qweight, sc, zeros, N, K, inv_s, y);
+    else
+      awq::gemv_w4a16_kernel<2><<<grid, awq::kGemvWarps * 32, 0, st>>>(
+          x, static_cast<int>(M), qweight, sc, zeros, N, K, inv_s, y);
+    return launch_status();
+  }
+  if (bits != 4) return AWQ_ERR_UNSUPPORTED;
+  if ((N + awq::kTcBM - 1) / awq::kTcBM > 65535) return AWQ_ERR_INVALID_ARG;
+  const __half* xop = x;
+  if (inv_s != nullptr) {
+    const size_t need = align256(static_cast<size_t>(M) * K * sizeof(__half));
+    if (!workspace || ws_bytes < need || !aligned16(workspace)) return AWQ_ERR_WORKSPACE;
+    __half* xs = static_cast<__half*>(workspace);
+    const int64_t n8 = M * K / 8;
+    awq::prescale_x_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, st>>>(x, inv_s, M,
+                                                                                   K, xs);
+    awq_status s = launch_status();
+    if (s != AWQ_OK) return s;
+    xop = xs;
+  }
+  awq::TcArgs args{};
+  args.M = M;
+  args.N = N;
+  args.N_pad = N;
+  args.K = K;
+  args.scales = sc;
+  args.zeros = zeros;
+  args.Y = y;
+  args.m_tiles = static_cast<int>((M + tc_bn_for(M) - 1) / tc_bn_for(M));
+  return launch_tc_bn<ASrc::kPacked4, Epi::kStoreY>(xop, M, qweight, N, args, st);
+}
+
+}  // extern "C"
