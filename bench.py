@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""W4A16 g128 GEMM on B200: GB/s at M = 1 (decode) and TFLOP/s at M = 2048 (prefill).
+
+One step of the headline workload is one decode GEMM (M = 1 token, 4-bit weights, groups of
+128) on each of the three decoder shapes [N, K] = [4096, 4096], [11008, 4096], [4096, 11008],
+with weights quantized by awq_quantize_pack on per-channel scales s = m^0.5 (m: lognormal
+channel magnitudes with 1% outliers x20). Inputs are already resident in HBM. The weights
+rotate through enough copies to exceed twice the L2, so every step streams from HBM; each
+step is replayed from a CUDA graph. `value` is the algorithmic bytes of all ranks' steps
+(codes + fp16 scales + uint8 zeros + X + Y) over the slowest rank's device time.
+
+The line also carries: the prefill GEMMs at M = 2048 on [28672, 8192], [8192, 28672] and
+[10240, 8192] (TFLOP/s, 2MNK per GEMM), the per-(shape, M) decode sweep, the dominant
+kernel's roofline fraction, an end-to-end figure through the Python binding with host
+buffers (copies inside the timed region), the CPU oracle on a bounded sample, and the SM
+clocks sampled during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "W4A16 g128 GEMM: GB/s at M=1, TFLOP/s at M=2048; % of B200 roofline"
+GROUP = 128
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def gemm_bytes(M, N, K, bits=4):
+    return N * K * bits // 8 + N * (K // GROUP) * 3 + 2 * M * K + 2 * M * N
+
+
+# ----------------------------------------------------------------------------- distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = [v for v in sm if v > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+class DecodeShape:
+    """One decode shape's rotating weight copies and its input/output buffers."""
+
+    def __init__(self, awq, N, K, m_max, l2_bytes, device):
+        W, mag, X = synth.decode_layer(N, K, m_max)
+        s = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(device)
+        Wd = torch.from_numpy(W).to(device)
+        base = awq.awq_quantize_pack(Wd, s, 4)
+        del Wd
+        per_copy = sum(t.numel() * t.element_size() for t in base)
+        self.copies = max(2, math.ceil(2 * l2_bytes / per_copy))
+        self.w = [base] + [tuple(t.clone() for t in base) for _ in range(self.copies - 1)]
+        self.N, self.K = N, K
+        self.X = torch.from_numpy(X).to(device)
+        self.Y = torch.empty(m_max, N, dtype=torch.float16, device=device)
+        self.Xh = torch.from_numpy(X).pin_memory()
+        self.Yh = torch.empty(m_max, N, dtype=torch.float16).pin_memory()
+
+    def call(self, awq, M, r, stream=None):
+        qw, sc, z = self.w[r % self.copies]
+        awq.awq_gemm_w4a16(self.X[:M], qw, sc, z, self.N, self.K, 4, out=self.Y[:M],
+                           stream=stream)
+
+
+def capture_steps(fn_per_step, n_graphs, stream):
+    graphs = []
+    for r in range(n_graphs):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn_per_step(r)
+        graphs.append(g)
+    return graphs
+
+
+def time_graphs(graphs, steps, warmup, stream, world):
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(steps):
+            graphs[i % len(graphs)].replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3   # seconds
+
+
+def cpu_oracle_sample(shapes, rows=512, repeats=2):
+    """The oracle (numpy, fp64) on a row slice of each decode shape at M = 1, one BLAS
+    thread. Returns (GB/s of algorithmic bytes, seconds, description)."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=1)
+    except ImportError:  # pragma: no cover
+        limiter = None
+    total_bytes, total_t = 0, 0.0
+    for (N, K) in shapes:
+        W, mag, X = synth.decode_layer(N, K, 1)
+        s = np.power(mag.astype(np.float64), 0.5).astype(np.float32)
+        Wr = W[:rows]
+        qw, sc, z = O.quantize_pack(Wr, s, 4, GROUP)
+        for _ in range(repeats):
+            t0 = time.perf_counter()
+            O.gemm_w4a16(X[:1], qw, sc, z, rows, K, 4, GROUP)
+            total_t += time.perf_counter() - t0
+            total_bytes += gemm_bytes(1, rows, K)
+    if limiter is not None:
+        limiter.unregister() if hasattr(limiter, "unregister") else None
+    desc = (f"oracle gemm_w4a16 (numpy fp64, 1 thread) at M=1 on the first {rows} rows of each "
+            f"decode shape, {repeats} calls each")
+    return total_bytes / total_t / 1e9, total_t, desc
+
+
+# ----------------------------------------------------------------------------- main arms
+
+def run_reference(args, world, rank):
+    """The CPU oracle timed as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle as O
+    shapes = synth.DECODE_SHAPES
+    rows = 256
+    prepared = []
+    for (N, K) in shapes:
+        W, mag, X = synth.decode_layer(N, K, 1)
+        s = np.power(mag.astype(np.float64), 0.5).astype(np.float32)
+        prepared.append((X[:1], O.quantize_pack(W[:rows], s, 4, GROUP), K))
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(limits=1)
+    except ImportError:  # pragma: no cover
+        pass
+    def step():
+        for X1, (qw, sc, z), K in prepared:
+            O.gemm_w4a16(X1, qw, sc, z, rows, K, 4, GROUP)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    step_bytes = sum(gemm_bytes(1, rows, K) for _, _, K in prepared)
+    v = step_bytes * args.steps / dt / 1e9
+    sample = (f"each step: oracle gemm_w4a16 at M=1 on the first {rows} rows of each decode "
+              f"shape {shapes} (numpy fp64, 1 thread)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "decode GEMM M=1 over [4096,4096], [11008,4096], [4096,11008] "
+                               "(W4 g128), row-sampled for the CPU oracle"},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_b200(args, world, rank, local):
+    import weight_only_int4_stats_b200 as awq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024)
+    pk = peaks()
+    stream = torch.cuda.Stream()
+
+    # ---- headline: decode GEMM at M = 1 over the three shapes
+    shapes = [DecodeShape(awq, N, K, 16, l2, dev) for (N, K) in synth.DECODE_SHAPES]
+    for sh in shapes:                     # first calls outside capture
+        sh.call(awq, 1, 0)
+    torch.cuda.synchronize()
+    n_graphs = max(sh.copies for sh in shapes)
+
+    def step(r):
+        for sh in shapes:
+            sh.call(awq, 1, r)
+    graphs = capture_steps(step, n_graphs, stream)
+    step_bytes = sum(gemm_bytes(1, sh.N, sh.K) for sh in shapes)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    dt = time_graphs(graphs, args.steps, args.warmup, stream, world)
+    clk = clocks.stop()
+    dt_max = max_over_ranks(dt, world)
+    value = step_bytes * args.steps * world / dt_max / 1e9
+    per_gpu = step_bytes * args.steps / dt / 1e9
+    launches = args.steps * len(shapes)
+    del graphs
+
+    # ---- decode sweep: each (shape, M) on its own
+    sweep = []
+    for sh in (shapes if args.only == "all" else []):
+        for M in synth.DECODE_M:
+            gs = capture_steps(lambda r, sh=sh, M=M: sh.call(awq, M, r), sh.copies, stream)
+            t = time_graphs(gs, 200, 10, stream, world)
+            b = gemm_bytes(M, sh.N, sh.K)
+            gbs = b * 200 / t / 1e9
+            sweep.append({"N": sh.N, "K": sh.K, "M": M, "us": t / 200 * 1e6, "GB/s": gbs,
+                          "TFLOP/s": 2 * M * sh.N * sh.K * 200 / t / 1e12,
+                          "frac_hbm": gbs / pk["hbm_gbs"]})
+            del gs
+
+    # ---- end to end through the binding with host buffers (no graph, copies timed)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = min(args.steps, 200)
+    h2d = sum(2 * sh.K for sh in shapes)
+    d2h = sum(2 * sh.N for sh in shapes)
+
+    def e2e_step(r):
+        for sh in shapes:
+            sh.X[:1].copy_(sh.Xh[:1], non_blocking=True)
+            sh.call(awq, 1, r)
+            sh.Yh[:1].copy_(sh.Y[:1], non_blocking=True)
+    with torch.cuda.stream(stream):
+        for r in range(3):
+            e2e_step(r)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for r in range(e2e_steps):
+            e2e_step(r)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+    e2e = {"value": step_bytes * e2e_steps * world / t_e2e / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "how": "python binding call per GEMM, pinned-host X copied in and Y copied out "
+                  "every step on the same stream, no graph"}
+    del shapes
+    torch.cuda.empty_cache()
+
+    # ---- prefill at M = 2048
+    prefill = []
+    for (N, K) in (synth.PREFILL_SHAPES if args.only != "decode" else []):
+        W, mag, X = synth.prefill_layer(N, K, 2048)
+        s = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(dev)
+        Wd = torch.from_numpy(W).to(dev)
+        del W
+        packs = [awq.awq_quantize_pack(Wd, s, 4)]
+        del Wd
+        packs.append(tuple(t.clone() for t in packs[0]))   # two copies > L2 with X
+        Xd = torch.from_numpy(X).to(dev)
+        Yd = torch.empty(2048, N, dtype=torch.float16, device=dev)
+        for p in packs:
+            awq.awq_gemm_w4a16(Xd, *p, N, K, 4, out=Yd)
+        torch.cuda.synchronize()
+        gs = capture_steps(lambda r: awq.awq_gemm_w4a16(Xd, *packs[r % 2], N, K, 4, out=Yd),
+                           2, stream)
+        iters = 20
+        t = time_graphs(gs, iters, 3, stream, world)
+        tfl = 2 * 2048 * N * K * iters / t / 1e12
+        prefill.append({"N": N, "K": K, "M": 2048, "ms": t / iters * 1e3, "TFLOP/s": tfl,
+                        "frac_tensor": tfl / pk["bf16_tflops"]})
+        del gs, packs, Xd, Yd
+        torch.cuda.empty_cache()
+    pf_flops = sum(2 * 2048 * p["N"] * p["K"] for p in prefill)
+    pf_time = sum(p["ms"] for p in prefill) / 1e3
+    pf_value = pf_flops / pf_time / 1e12 if prefill else None
+
+    if rank != 0:
+        return
+    cpu_gbs, cpu_t, cpu_desc = (cpu_oracle_sample(synth.DECODE_SHAPES) if args.only == "all"
+                                else (None, None, "skipped (--only)"))
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt_max / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {
+            "workload": "decode GEMM, M=1, W4 g128, [N,K] in [4096,4096], [11008,4096], "
+                        "[4096,11008]; one GEMM per shape per step",
+            "inputs": "weights rotate through copies totalling > 2x L2 (L2 not flushed)",
+            "replay": "CUDA graph per step",
+            "parallelism": f"replicas x{world} (no data-path collective)",
+        },
+        "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": per_gpu / pk["hbm_gbs"], "traffic": None,
+                     "kernel": "gemv_w4a16_kernel", "peak_source": pk["source"],
+                     "frac_of_8TBps_nominal": per_gpu / 8000.0},
+        "prefill": {"metric": "TFLOP/s at M=2048", "value": pf_value, "unit": "TFLOP/s",
+                    "per_shape": prefill, "peak": pk["bf16_tflops"],
+                    "frac": pf_value / pk["bf16_tflops"] if prefill else None,
+                    "kernel": "tc_gemm_kernel"},
+        "sweep": sweep,
+        "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": cpu_desc, "seconds": cpu_t},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--only", choices=["all", "decode", "prefill"], default="all",
+                    help="run one section only (used by the profiling commands)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_b200(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

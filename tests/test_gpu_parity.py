@@ -3,8 +3,15 @@
 Bars: bit-exact for integer work (codes, zeros, chosen grid index) and for values that are
 exact by construction (fp64-accumulated act_stats, the fp16 scales); relative Frobenius
 error <= 2e-3 for GEMM outputs (fp32 accumulation, fp16 output, against the fp64 oracle on
-the dequantized weights); search losses within 1e-4 relative and the chosen grid point
-equal to the oracle's unless the oracle itself rates the two within 1e-5 (a near tie).
+the dequantized weights).
+
+Search losses: the GPU evaluates ||E X^T||^2 with the error operand E rounded to fp16, a
+relative perturbation of at most u = 2^-11 per element. When one input channel dominates
+every output (an outlier channel), that perturbation does not average out over tokens and a
+loss can move by up to about 2u = 2^-10 relative; with many rows and tokens it averages
+down (observed ~1e-6 on the 512x512 layer). So losses must agree within 2^-10, and the
+chosen grid point must equal the oracle's unless the oracle rates the two within 2^-10 of
+each other (a near tie, where the fp16 rounding can legitimately swap them).
 """
 import numpy as np
 import pytest
@@ -16,8 +23,8 @@ import synth
 pytestmark = pytest.mark.gpu
 
 GEMM_RTOL = 2e-3
-LOSS_RTOL = 1e-4
-NEAR_TIE = 1e-5
+LOSS_RTOL = 2.0 ** -10
+NEAR_TIE = 2.0 ** -10
 
 
 @pytest.fixture(scope="module")
