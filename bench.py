@@ -340,33 +340,35 @@ def run_b200(args, world, rank, local):
     del shapes
     torch.cuda.empty_cache()
 
-    # ---- prefill at M = 2048
+    # ---- prefill at M = 2048 (4-bit on the three shapes, then the 3-bit variant)
     prefill = []
-    for (N, K) in (synth.PREFILL_SHAPES if args.only != "decode" else []):
+    pf_cases = [(N, K, 4) for (N, K) in synth.PREFILL_SHAPES] + [(*synth.PREFILL_SHAPES[0], 3)]
+    for (N, K, bits) in (pf_cases if args.only != "decode" else []):
         W, mag, X = synth.prefill_layer(N, K, 2048)
         s = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(dev)
         Wd = torch.from_numpy(W).to(dev)
         del W
-        packs = [awq.awq_quantize_pack(Wd, s, 4)]
+        packs = [awq.awq_quantize_pack(Wd, s, bits)]
         del Wd
         packs.append(tuple(t.clone() for t in packs[0]))   # two copies > L2 with X
         Xd = torch.from_numpy(X).to(dev)
         Yd = torch.empty(2048, N, dtype=torch.float16, device=dev)
         for p in packs:
-            awq.awq_gemm_w4a16(Xd, *p, N, K, 4, out=Yd)
+            awq.awq_gemm_w4a16(Xd, *p, N, K, bits, out=Yd)
         torch.cuda.synchronize()
-        gs = capture_steps(lambda r: awq.awq_gemm_w4a16(Xd, *packs[r % 2], N, K, 4, out=Yd),
+        gs = capture_steps(lambda r: awq.awq_gemm_w4a16(Xd, *packs[r % 2], N, K, bits, out=Yd),
                            2, stream)
         iters = 20
         t = time_graphs(gs, iters, 3, stream, world)
         tfl = 2 * 2048 * N * K * iters / t / 1e12
-        prefill.append({"N": N, "K": K, "M": 2048, "ms": t / iters * 1e3, "TFLOP/s": tfl,
-                        "frac_tensor": tfl / pk["bf16_tflops"]})
+        prefill.append({"N": N, "K": K, "M": 2048, "bits": bits, "ms": t / iters * 1e3,
+                        "TFLOP/s": tfl, "frac_tensor": tfl / pk["bf16_tflops"]})
         del gs, packs, Xd, Yd
         torch.cuda.empty_cache()
-    pf_flops = sum(2 * 2048 * p["N"] * p["K"] for p in prefill)
-    pf_time = sum(p["ms"] for p in prefill) / 1e3
-    pf_value = pf_flops / pf_time / 1e12 if prefill else None
+    pf4 = [p for p in prefill if p["bits"] == 4]
+    pf_flops = sum(2 * 2048 * p["N"] * p["K"] for p in pf4)
+    pf_time = sum(p["ms"] for p in pf4) / 1e3
+    pf_value = pf_flops / pf_time / 1e12 if pf4 else None
 
     if rank != 0:
         return

@@ -161,12 +161,21 @@ def test_gemm_decode_full_shapes(awq, N, K):
         _check_gemm(awq, X[:M], qw, sc, z, N, K)
 
 
+@pytest.mark.parametrize("bits", [4, 3])
 @pytest.mark.parametrize("M", [17, 32, 33, 64, 65, 128, 200, 256, 300, 600])
 @pytest.mark.parametrize("N,K", [(256, 256), (200, 384), (384, 1024)])
-def test_gemm_tensor_core(awq, M, N, K):
+def test_gemm_tensor_core(awq, M, N, K, bits):
     W, X, m = rand_layer(M * 17 + N + K, N, K, M)
-    qw, sc, z = _packed(W, np.sqrt(m).astype(np.float32))
-    _check_gemm(awq, X, qw, sc, z, N, K)
+    qw, sc, z = _packed(W, np.sqrt(m).astype(np.float32), bits)
+    _check_gemm(awq, X, qw, sc, z, N, K, bits)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_gemm_3bit_decode_sizes(awq, M):
+    N, K = 320, 768
+    W, X, m = rand_layer(M + 900, N, K, M)
+    qw, sc, z = _packed(W, np.sqrt(m).astype(np.float32), 3)
+    _check_gemm(awq, X, qw, sc, z, N, K, 3)
 
 
 def test_gemm_tensor_core_inv_s(awq):
@@ -186,14 +195,15 @@ def test_gemm_batched_full_shapes(awq, N, K):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("N,K", synth.PREFILL_SHAPES)
-def test_gemm_prefill_full_shape_sampled(awq, N, K):
+@pytest.mark.parametrize("N,K,bits", [(n, k, 4) for (n, k) in synth.PREFILL_SHAPES] +
+                         [(synth.PREFILL_SHAPES[0][0], synth.PREFILL_SHAPES[0][1], 3)])
+def test_gemm_prefill_full_shape_sampled(awq, N, K, bits):
     # Full-size launch (M = 2048); the oracle checks 16 sampled token rows against all N.
     W, m, X = synth.prefill_layer(N, K, 2048)
-    qw, sc, z = _packed(W, np.power(m.astype(np.float64), 0.5).astype(np.float32))
+    qw, sc, z = _packed(W, np.power(m.astype(np.float64), 0.5).astype(np.float32), bits)
     rows = np.random.default_rng(0).choice(2048, 16, replace=False)
     rows.sort()
-    _check_gemm(awq, X, qw, sc, z, N, K, rows=rows)
+    _check_gemm(awq, X, qw, sc, z, N, K, bits, rows=rows)
     torch.cuda.empty_cache()
 
 
@@ -293,3 +303,38 @@ def test_search_full_decoder_layer_sampled_rows(awq):
     np.testing.assert_array_equal(best_s.cpu().numpy(), table[b])
     del acts, X
     torch.cuda.empty_cache()
+
+
+# ----------------------------------------------------------------------------- stream ordering
+
+def test_decode_right_after_quantize_on_same_stream(awq):
+    # The decode kernel may start before the previous kernel on the stream has finished
+    # (programmatic dependent launch); the packed weights written by that kernel must still
+    # be the ones it reads.
+    N, K = 2048, 1024
+    W, X, m = rand_layer(404, N, K, 1)
+    s = np.sqrt(m).astype(np.float32)
+    Wd, sd, Xd = cu(W), cu(s), cu(X)
+    for _ in range(3):
+        qw, sc, z = awq.awq_quantize_pack(Wd, sd, 4)
+        Y = awq.awq_gemm_w4a16(Xd, qw, sc, z, N, K)
+    oq, osc, oz = O.quantize_pack(W, s, 4, 128)
+    want = O.gemm_w4a16(X, oq, osc, oz, N, K, 4, 128)
+    assert rel_fro(Y.float().cpu().numpy(), want) <= GEMM_RTOL
+
+
+def test_decode_chain_output_feeds_next_input(awq):
+    # Y1 = X W1^T, Y2 = Y1 W2^T back to back: the second call's activations are the first
+    # call's output.
+    K1, N1, N2 = 1024, 2048, 512
+    W1, X, m = rand_layer(505, N1, K1, 1)
+    W2, _, _ = rand_layer(506, N2, N1, 1)
+    p1 = O.quantize_pack(W1, None, 4, 128)
+    p2 = O.quantize_pack(W2, None, 4, 128)
+    d1 = [cu(a) for a in p1]
+    d2 = [cu(a) for a in p2]
+    Y1 = awq.awq_gemm_w4a16(cu(X), *d1, N1, K1)
+    Y2 = awq.awq_gemm_w4a16(Y1, *d2, N2, N1)
+    o1 = O.gemm_w4a16(X, *p1, N1, K1, 4, 128).astype(np.float16)
+    o2 = O.gemm_w4a16(o1, *p2, N2, N1, 4, 128)
+    assert rel_fro(Y2.float().cpu().numpy(), o2) <= GEMM_RTOL

@@ -26,8 +26,6 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 size_t align256(size_t v) { return (v + 255) & ~size_t{255}; }
 
-awq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA; }
-
 awq_status launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
@@ -104,9 +102,13 @@ awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_ro
     if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a_rows, args.K, awq::kTcBM,
                       awq::kTcBK, true))
       return AWQ_ERR_CUDA;
-  } else {
+  } else if (kA == ASrc::kPacked4) {
     if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a_rows, args.K / 8,
                       awq::kTcBM, awq::kTcBK / 8, false))
+      return AWQ_ERR_CUDA;
+  } else {   // 3-bit: one 128-k group = 12 words (48 bytes) per row per load
+    if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a_rows, 3 * args.K / 32,
+                      awq::kTcBM, 12, false))
       return AWQ_ERR_CUDA;
   }
   dim3 grid(static_cast<unsigned>((M + BN - 1) / BN),
@@ -122,6 +124,67 @@ awq_status launch_tc_bn(const __half* Xop, int64_t M, const void* Aop, int64_t a
   if (M <= 64) return launch_tc<64, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
   if (M <= 128) return launch_tc<128, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
   return launch_tc<256, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
+}
+
+// Streaming decode GEMM (M <= 16, 4-bit): returns AWQ_ERR_UNSUPPORTED when the shape does
+// not suit it (the caller then uses the register-streaming kernel).
+constexpr int kSmemLimit = 232448;   // 227 KB per CTA on sm_100
+
+template <int kNTiles>
+awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweight,
+                              const __half* scales, const uint8_t* zeros, int64_t N, int64_t K,
+                              const float* inv_s, __half* y, cudaStream_t st) {
+  if (N % 16 != 0) return AWQ_ERR_UNSUPPORTED;
+  awq::G2Smem lay;
+  lay.x_bytes = static_cast<int>(round_up(M * K * 2, 128));
+  int slots = 8;
+  while (slots >= 2) {
+    lay.slots = slots;
+    if (lay.template total<kNTiles>() <= kSmemLimit) break;
+    slots /= 2;
+  }
+  if (slots < 2) return AWQ_ERR_UNSUPPORTED;
+  const int smem = lay.template total<kNTiles>();
+  static bool attr_set[kMaxDevices] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
+  auto kern = awq::gemv_stream_kernel<kNTiles>;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+        cudaSuccess)
+      return AWQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, awq::kG2Threads, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return AWQ_ERR_CUDA;
+  const int64_t tiles = N / 16;
+  const int64_t resident = static_cast<int64_t>(num_sms()) * per_sm;
+  const unsigned grid = static_cast<unsigned>(tiles < resident ? tiles : resident);
+  CUtensorMap tw, ts, tz;
+  if (!make_tmap_2d(&tw, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, 16, awq::kG2KC / 8,
+                    false) ||
+      !make_tmap_2d(&ts, scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K / awq::kGroup, N,
+                    awq::kG2Warps, 16, false) ||
+      !make_tmap_2d(&tz, zeros, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / awq::kGroup, N,
+                    awq::kG2Warps, 16, false))
+    return AWQ_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(awq::kG2Threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int m32 = static_cast<int>(M);
+  if (cudaLaunchKernelEx(&cfg, kern, tw, ts, tz, qweight, x, m32, N, K, inv_s, y, lay) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  return launch_status();
 }
 
 int tc_bn_for(int64_t M) { return M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
@@ -328,6 +391,9 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
   __half* y = reinterpret_cast<__half*>(Y);
 
   if (M <= 16 && bits == 4) {
+    awq_status r = M <= 8 ? launch_gemv_stream<1>(x, M, qweight, sc, zeros, N, K, inv_s, y, st)
+                          : launch_gemv_stream<2>(x, M, qweight, sc, zeros, N, K, inv_s, y, st);
+    if (r != AWQ_ERR_UNSUPPORTED) return r;
     const unsigned grid = static_cast<unsigned>((N + awq::kGemvRows - 1) / awq::kGemvRows);
     if (M <= 8)
       awq::gemv_w4a16_kernel<1><<<grid, awq::kGemvWarps * 32, 0, st>>>(
@@ -337,7 +403,6 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
           x, static_cast<int>(M), qweight, sc, zeros, N, K, inv_s, y);
     return launch_status();
   }
-  if (bits != 4) return AWQ_ERR_UNSUPPORTED;
   if ((N + awq::kTcBM - 1) / awq::kTcBM > 65535) return AWQ_ERR_INVALID_ARG;
   const __half* xop = x;
   if (inv_s != nullptr) {
@@ -360,6 +425,7 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
   args.zeros = zeros;
   args.Y = y;
   args.m_tiles = static_cast<int>((M + tc_bn_for(M) - 1) / tc_bn_for(M));
+  if (bits == 3) return launch_tc_bn<ASrc::kPacked3, Epi::kStoreY>(xop, M, qweight, N, args, st);
   return launch_tc_bn<ASrc::kPacked4, Epi::kStoreY>(xop, M, qweight, N, args, st);
 }
 

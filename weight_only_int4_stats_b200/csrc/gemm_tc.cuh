@@ -29,24 +29,31 @@ namespace awq {
 constexpr int kTcBM = 128;      // weight rows per tile (MMA M)
 constexpr int kTcBK = 64;       // K per stage: one 128-byte swizzle atom of fp16
 constexpr int kTcStages = 4;
-constexpr int kTcThreads = 192; // 6 warps
+constexpr int kTcBuilders = 8;  // A-builder / epilogue warps
+constexpr int kTcThreads = (2 + kTcBuilders) * 32;
+constexpr int kTcPk3Slots = 2;  // 3-bit packed ring: one 128-k group (48 B per row) per slot
 
-enum class ASrc : int { kPacked4 = 0, kFp16 = 1 };
+enum class ASrc : int { kPacked4 = 0, kPacked3 = 1, kFp16 = 2 };
 enum class Epi : int { kStoreY = 0, kRowSumSq = 1 };
 
 template <int BN, ASrc kA>
 struct TcLayout {
   static constexpr int kXBytes = BN * kTcBK * 2;
   static constexpr int kABytes = kTcBM * kTcBK * 2;
-  static constexpr int kPBytes = (kA == ASrc::kPacked4) ? kTcBM * kTcBK / 2 : 0;
+  // packed source per stage (4-bit) or per ring slot (3-bit, one group of 128 k)
+  static constexpr int kPBytes = kA == ASrc::kPacked4 ? kTcBM * kTcBK / 2
+                               : kA == ASrc::kPacked3 ? kTcBM * 48 : 0;
+  static constexpr int kPSlots = kA == ASrc::kPacked3 ? kTcPk3Slots : kTcStages;
   static constexpr int kXOff = 0;
   static constexpr int kAOff = kXOff + kTcStages * kXBytes;
   static constexpr int kPOff = kAOff + kTcStages * kABytes;
-  static constexpr int kBarOff = kPOff + kTcStages * kPBytes;
-  // full[S], empty[S], built[S], acc_full, tmem slot
-  static constexpr int kBytes = kBarOff + (3 * kTcStages + 1) * 8 + 16;
+  static constexpr int kRedOff = kPOff + kPSlots * kPBytes;          // 128 doubles
+  static constexpr int kBarOff = kRedOff + kTcBM * 8;
+  // full[S], empty[S], built[S], pfull[2], pempty[2], acc_full, tmem slot
+  static constexpr int kBytes = kBarOff + (3 * kTcStages + 2 * kTcPk3Slots + 1) * 8 + 16;
   static constexpr int kSmem = kBytes + 1024;   // slack for 1024-byte alignment
-  static constexpr uint32_t kTxBytes = kXBytes + (kA == ASrc::kFp16 ? kABytes : kPBytes);
+  static constexpr uint32_t kTxBytes =
+      kXBytes + (kA == ASrc::kFp16 ? kABytes : kA == ASrc::kPacked4 ? kPBytes : 0);
   static constexpr uint32_t kTmemCols = BN;     // fp32 accumulator columns (power of 2)
 };
 
@@ -62,7 +69,7 @@ struct TcArgs {
   int m_tiles;
 };
 
-// Dequantize one packed word (8 consecutive k) to four fp16 pairs (q - z) * sc.
+// Dequantize one 4-bit packed word (8 consecutive k) to four fp16 pairs (q - z) * sc.
 __device__ __forceinline__ uint4 dequant_word_scaled(uint32_t w, __half2 bias_lo,
                                                      __half2 bias_hi, __half2 sc2) {
   const __half2 sixteenth = __float2half2_rn(0.0625f);
@@ -79,6 +86,22 @@ __device__ __forceinline__ uint4 dequant_word_scaled(uint32_t w, __half2 bias_lo
   return o;
 }
 
+// 3-bit: the fp16 pair (q - z) * sc for k-offsets (2e, 2e+1) of chunk i (k = 8i..8i+7) of a
+// 32-k block whose low-bit words are w0 (offsets 0..15) / w1 (16..31) and whose bit-2 word,
+// pre-shifted left by 2, is w2s.
+template <int kI, int kE>
+__device__ __forceinline__ uint32_t dequant3_pair(uint32_t w0, uint32_t w1, uint32_t w2s,
+                                                  __half2 bias_lo, __half2 sc2) {
+  constexpr int pp = 4 * (kI & 1) + kE;     // 2-bit field of the pair inside its low word
+  constexpr int hb = 4 * kI + kE;           // bit of the pair inside the bit-2 word
+  const uint32_t wlo = (kI < 2) ? w0 : w1;
+  const uint32_t lo = lop3_and_or(wlo >> (2 * pp), 0x00030003u, 0x64006400u);
+  uint32_t v;
+  // (w2s >> hb) & 0x00040004 | lo
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(v) : "r"(w2s >> hb), "r"(0x00040004u), "r"(lo));
+  return h2_as_u32(__hmul2(__hsub2(u32_as_h2(v), bias_lo), sc2));
+}
+
 // Byte offset of 16-byte chunk c (k = 8c..8c+7) of row r in a 64-wide fp16 tile stored in
 // the 128-byte swizzled K-major layout (8-row atoms of 1024 bytes).
 __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
@@ -90,14 +113,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                    const __grid_constant__ CUtensorMap tmap_a, const TcArgs args) {
   using L = TcLayout<BN, kA>;
+  constexpr bool kPacked = kA != ASrc::kFp16;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* empty = full + kTcStages;
   uint64_t* built = empty + kTcStages;
-  uint64_t* acc_full = built + kTcStages;
+  uint64_t* pfull = built + kTcStages;
+  uint64_t* pempty = pfull + kTcPk3Slots;
+  uint64_t* acc_full = pempty + kTcPk3Slots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  double* red = reinterpret_cast<double*>(smem + L::kRedOff);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -111,7 +138,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int s = 0; s < kTcStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&built[s], 128);
+      mbar_init(&built[s], kTcBuilders * 32);
+    }
+    for (int s = 0; s < kTcPk3Slots; ++s) {
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pempty[s], kTcBuilders * 32);
     }
     mbar_init(acc_full, 1);
     fence_barrier_init();
@@ -133,6 +164,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % kTcStages;
         const uint32_t ph = (kb / kTcStages) & 1;
+        if (kA == ASrc::kPacked3 && (kb & 1) == 0) {
+          const int pk = kb >> 1, ps = pk % kTcPk3Slots;
+          if (!mbar_wait(&pempty[ps], ((pk / kTcPk3Slots) & 1) ^ 1)) break;
+          mbar_arrive_expect_tx(&pfull[ps], L::kPBytes);
+          tma_load_2d(smem + L::kPOff + ps * L::kPBytes, &tmap_a, &pfull[ps], pk * 12,
+                      static_cast<int32_t>(row0));
+        }
         if (!mbar_wait(&empty[s], ph ^ 1)) break;
         mbar_arrive_expect_tx(&full[s], L::kTxBytes);
         tma_load_2d(smem + L::kXOff + s * L::kXBytes, &tmap_x, &full[s], kb * kTcBK,
@@ -140,7 +178,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (kA == ASrc::kFp16)
           tma_load_2d(smem + L::kAOff + s * L::kABytes, &tmap_a, &full[s], kb * kTcBK,
                       static_cast<int32_t>(row0));
-        else
+        else if (kA == ASrc::kPacked4)
           tma_load_2d(smem + L::kPOff + s * L::kPBytes, &tmap_a, &full[s], kb * (kTcBK / 8),
                       static_cast<int32_t>(row0));
       }
@@ -154,15 +192,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int s = kb % kTcStages;
         const uint32_t ph = (kb / kTcStages) & 1;
         ok = mbar_wait(&full[s], ph);
-        if (ok && kA == ASrc::kPacked4) ok = mbar_wait(&built[s], ph);
+        if (ok && kPacked) ok = mbar_wait(&built[s], ph);
         if (!ok) break;
         tc_fence_after();
         const uint32_t a_base = smem_u32(smem + L::kAOff + s * L::kABytes);
         const uint32_t x_base = smem_u32(smem + L::kXOff + s * L::kXBytes);
 #pragma unroll
         for (int kk = 0; kk < kTcBK / 16; ++kk) {
-          tc_mma_f16(tmem_d, sw128_kmajor_desc(a_base + kk * 32), sw128_kmajor_desc(x_base + kk * 32),
-                     idesc, (kb | kk) != 0 ? 1u : 0u);
+          tc_mma_f16(tmem_d, sw128_kmajor_desc(a_base + kk * 32),
+                     sw128_kmajor_desc(x_base + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
         }
         tc_commit(&empty[s]);
       }
@@ -170,85 +208,103 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ A builders
-    const int t = threadIdx.x - 64;   // 0..127
+    const int t = threadIdx.x - 64;            // 0..255
+    const int r = t >> 1, h = t & 1;           // tile row, 32-k half of the 64-k stage
+    const int64_t n = row0 + r;
+    const int64_t N = args.N;
     bool ok = true;
-    if (kA == ASrc::kPacked4) {
-      const int64_t N = args.N;
-      const int rA = t >> 1, rB = rA + 64;
-      const int64_t nA = row0 + rA, nB = row0 + rB;
-      __half2 loA, hiA, scA, loB, hiB, scB;
+    if (kPacked) {
+      __half2 lo, hi, sc;
       for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % kTcStages;
         const uint32_t ph = (kb / kTcStages) & 1;
-        if ((kb & 1) == 0) {   // new group of 128: this thread's two rows' zero and scale
+        if ((kb & 1) == 0) {   // new group of 128: this row's zero point and scale
           const int64_t g = kb >> 1;
-          const uint32_t zA = nA < N ? args.zeros[g * N + nA] : 0u;
-          const uint32_t zB = nB < N ? args.zeros[g * N + nB] : 0u;
-          const __half sA = nA < N ? args.scales[g * N + nA] : __float2half(0.0f);
-          const __half sB = nB < N ? args.scales[g * N + nB] : __float2half(0.0f);
-          loA = u32_as_h2((0x6400u | zA) * 0x00010001u);
-          hiA = __hneg2(u32_as_h2((0x5400u | (zA << 4)) * 0x00010001u));
-          loB = u32_as_h2((0x6400u | zB) * 0x00010001u);
-          hiB = __hneg2(u32_as_h2((0x5400u | (zB << 4)) * 0x00010001u));
-          scA = __half2half2(sA);
-          scB = __half2half2(sB);
+          const uint32_t z = n < N ? args.zeros[g * N + n] : 0u;
+          const __half sv = n < N ? args.scales[g * N + n] : __float2half(0.0f);
+          lo = u32_as_h2((0x6400u | z) * 0x00010001u);
+          hi = __hneg2(u32_as_h2((0x5400u | (z << 4)) * 0x00010001u));
+          sc = __half2half2(sv);
         }
-        ok = mbar_wait(&full[s], ph) && mbar_wait(&empty[s], ph ^ 1);
-        ok = __all_sync(0xffffffffu, ok);   // keep the warp converged for .aligned ops
+        bool got = mbar_wait(&full[s], ph) && mbar_wait(&empty[s], ph ^ 1);
+        const int pk = kb >> 1, ps = pk % kTcPk3Slots;
+        if (kA == ASrc::kPacked3 && got) got = mbar_wait(&pfull[ps], (pk / kTcPk3Slots) & 1);
+        ok = __all_sync(0xffffffffu, got);   // keep the warp converged for .aligned ops
         if (!ok) break;
-        const uint8_t* ptile = smem + L::kPOff + s * L::kPBytes;
         uint8_t* atile = smem + L::kAOff + s * L::kABytes;
-#pragma unroll
-        for (int pass = 0; pass < 2; ++pass) {
-          const int q = t + 128 * pass;          // 16-byte chunk of the packed tile
-          const int r = q >> 1, h = q & 1;        // row, which 32-k half of the 64
-          const uint4 pw = *reinterpret_cast<const uint4*>(ptile + q * 16);
-          const __half2 lo = pass ? loB : loA, hi = pass ? hiB : hiA, sc = pass ? scB : scA;
+        if (kA == ASrc::kPacked4) {
+          const uint8_t* ptile = smem + L::kPOff + s * L::kPBytes;
+          const uint4 pw = *reinterpret_cast<const uint4*>(ptile + t * 16);   // row r, half h
           const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const uint4 o = dequant_word_scaled(words[i], lo, hi, sc);
             *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + i)) = o;
           }
+        } else {
+          const uint32_t* pw = reinterpret_cast<const uint32_t*>(
+              smem + L::kPOff + ps * L::kPBytes + r * 48 + 12 * (2 * (kb & 1) + h));
+          const uint32_t w0 = pw[0], w1 = pw[1], w2s = pw[2] << 2;
+          uint4 o;
+#define AWQ_DQ3_CHUNK(I)                                                   \
+  o.x = dequant3_pair<I, 0>(w0, w1, w2s, lo, sc);                         \
+  o.y = dequant3_pair<I, 1>(w0, w1, w2s, lo, sc);                         \
+  o.z = dequant3_pair<I, 2>(w0, w1, w2s, lo, sc);                         \
+  o.w = dequant3_pair<I, 3>(w0, w1, w2s, lo, sc);                         \
+  *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + I)) = o;
+          AWQ_DQ3_CHUNK(0)
+          AWQ_DQ3_CHUNK(1)
+          AWQ_DQ3_CHUNK(2)
+          AWQ_DQ3_CHUNK(3)
+#undef AWQ_DQ3_CHUNK
+          if (kb & 1) mbar_arrive(&pempty[ps]);   // both stages of the group are built
         }
         fence_proxy_async_smem();
         mbar_arrive(&built[s]);
       }
     }
     // ------------------------------------------------------------------ epilogue
+    // Warp w reads TMEM lane quarter (w % 4) -- the only one it may access -- and half of
+    // the BN token columns; the two halves of a row's sum of squares meet in shared memory.
     if (ok) ok = mbar_wait(acc_full, 0);
     ok = __all_sync(0xffffffffu, ok);
+    const int wq = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = 32 * wq + lane;
+    const int64_t arow = row0 + row;
+    double sumsq = 0.0;
     if (ok) {
       tc_fence_after();
-      const int wq = warp & 3;                 // TMEM lane quarter this warp may access
-      const int row = 32 * wq + lane;          // row inside the tile
-      const int64_t arow = row0 + row;
-      double sumsq = 0.0;
+      constexpr int kHalf = BN / 2;
 #pragma unroll 1
-      for (int cb = 0; cb < BN / 32; ++cb) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(32 * wq) << 16) + cb * 32, v);
+      for (int cb = 0; cb < kHalf; cb += 16) {
+        uint32_t v[16];
+        const int col = half * kHalf + cb;
+        tmem_ld_32x32b_x16(tmem_d + (static_cast<uint32_t>(32 * wq) << 16) + col, v);
         tmem_ld_wait();
         if (kEpi == Epi::kStoreY) {
           if (arow < args.N) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int64_t m = m0 + cb * 32 + j;
+            for (int j = 0; j < 16; ++j) {
+              const int64_t m = m0 + col + j;
               if (m < args.M) args.Y[m * args.N + arow] = __float2half_rn(__uint_as_float(v[j]));
             }
           }
         } else {
           float part = 0.0f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const float f = __uint_as_float(v[j]);
             part = fmaf(f, f, part);
           }
           sumsq += static_cast<double>(part);
         }
       }
-      if (kEpi == Epi::kRowSumSq)
-        args.row_part[arow * args.m_tiles + m_tile] = sumsq;
+    }
+    if (kEpi == Epi::kRowSumSq) {
+      if (half == 1) red[row] = sumsq;
+      named_bar_sync(1, kTcBuilders * 32);
+      if (half == 0 && ok) args.row_part[arow * args.m_tiles + m_tile] = sumsq + red[row];
     }
   }
 
