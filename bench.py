@@ -6,7 +6,7 @@ One step of the headline workload is one decode GEMM (M = 1 token, 4-bit weights
 with weights quantized by awq_quantize_pack on per-channel scales s = m^0.5 (m: lognormal
 channel magnitudes with 1% outliers x20). Inputs are already resident in HBM. The weights
 rotate through enough copies to exceed twice the L2, so every step streams from HBM; each
-step is replayed from a CUDA graph. `value` is the algorithmic bytes of all ranks' steps
+run of steps is captured in one CUDA graph. `value` is the algorithmic bytes of all ranks' steps
 (codes + fp16 scales + uint8 zeros + X + Y) over the slowest rank's device time.
 
 The line also carries: the prefill GEMMs at M = 2048 on [28672, 8192], [8192, 28672] and
@@ -164,20 +164,23 @@ class DecodeShape:
                            stream=stream)
 
 
-def capture_steps(fn_per_step, n_graphs, stream):
-    graphs = []
-    for r in range(n_graphs):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
+def capture_run(fn_per_step, first, count, stream):
+    """One CUDA graph holding `count` consecutive steps (step r uses rotation index r), so
+    the kernels run back to back without a graph launch between them."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for r in range(first, first + count):
             fn_per_step(r)
-        graphs.append(g)
-    return graphs
+    return g
 
 
-def time_graphs(graphs, steps, warmup, stream, world):
+def time_steps(fn_per_step, steps, warmup, stream, world):
+    """Warm-up graph of `warmup` steps, then a graph of exactly `steps` steps timed with
+    CUDA events on `stream`, with a barrier and a device synchronisation on both sides."""
+    gw = capture_run(fn_per_step, 0, warmup, stream)
+    gt = capture_run(fn_per_step, warmup, steps, stream)
     with torch.cuda.stream(stream):
-        for i in range(warmup):
-            graphs[i % len(graphs)].replay()
+        gw.replay()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -185,12 +188,12 @@ def time_graphs(graphs, steps, warmup, stream, world):
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for i in range(steps):
-            graphs[i % len(graphs)].replay()
+        gt.replay()
         e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
+    del gw, gt
     return e0.elapsed_time(e1) / 1e3   # seconds
 
 
@@ -280,36 +283,30 @@ def run_b200(args, world, rank, local):
     for sh in shapes:                     # first calls outside capture
         sh.call(awq, 1, 0)
     torch.cuda.synchronize()
-    n_graphs = max(sh.copies for sh in shapes)
-
     def step(r):
         for sh in shapes:
             sh.call(awq, 1, r)
-    graphs = capture_steps(step, n_graphs, stream)
     step_bytes = sum(gemm_bytes(1, sh.N, sh.K) for sh in shapes)
 
     clocks = ClockSampler(local)
     clocks.start()
-    dt = time_graphs(graphs, args.steps, args.warmup, stream, world)
+    dt = time_steps(step, args.steps, args.warmup, stream, world)
     clk = clocks.stop()
     dt_max = max_over_ranks(dt, world)
     value = step_bytes * args.steps * world / dt_max / 1e9
     per_gpu = step_bytes * args.steps / dt / 1e9
     launches = args.steps * len(shapes)
-    del graphs
 
     # ---- decode sweep: each (shape, M) on its own
     sweep = []
     for sh in (shapes if args.only == "all" else []):
         for M in synth.DECODE_M:
-            gs = capture_steps(lambda r, sh=sh, M=M: sh.call(awq, M, r), sh.copies, stream)
-            t = time_graphs(gs, 200, 10, stream, world)
+            t = time_steps(lambda r, sh=sh, M=M: sh.call(awq, M, r), 200, 10, stream, world)
             b = gemm_bytes(M, sh.N, sh.K)
             gbs = b * 200 / t / 1e9
             sweep.append({"N": sh.N, "K": sh.K, "M": M, "us": t / 200 * 1e6, "GB/s": gbs,
                           "TFLOP/s": 2 * M * sh.N * sh.K * 200 / t / 1e12,
                           "frac_hbm": gbs / pk["hbm_gbs"]})
-            del gs
 
     # ---- end to end through the binding with host buffers (no graph, copies timed)
     e0 = torch.cuda.Event(enable_timing=True)
@@ -356,14 +353,13 @@ def run_b200(args, world, rank, local):
         for p in packs:
             awq.awq_gemm_w4a16(Xd, *p, N, K, bits, out=Yd)
         torch.cuda.synchronize()
-        gs = capture_steps(lambda r: awq.awq_gemm_w4a16(Xd, *packs[r % 2], N, K, bits, out=Yd),
-                           2, stream)
         iters = 20
-        t = time_graphs(gs, iters, 3, stream, world)
+        t = time_steps(lambda r: awq.awq_gemm_w4a16(Xd, *packs[r % 2], N, K, bits, out=Yd),
+                       iters, 3, stream, world)
         tfl = 2 * 2048 * N * K * iters / t / 1e12
         prefill.append({"N": N, "K": K, "M": 2048, "bits": bits, "ms": t / iters * 1e3,
                         "TFLOP/s": tfl, "frac_tensor": tfl / pk["bf16_tflops"]})
-        del gs, packs, Xd, Yd
+        del packs, Xd, Yd
         torch.cuda.empty_cache()
     pf4 = [p for p in prefill if p["bits"] == 4]
     pf_flops = sum(2 * 2048 * p["N"] * p["K"] for p in pf4)
@@ -383,7 +379,8 @@ def run_b200(args, world, rank, local):
             "workload": "decode GEMM, M=1, W4 g128, [N,K] in [4096,4096], [11008,4096], "
                         "[4096,11008]; one GEMM per shape per step",
             "inputs": "weights rotate through copies totalling > 2x L2 (L2 not flushed)",
-            "replay": "CUDA graph per step",
+            "replay": "warm-up steps and the K timed steps each captured in one CUDA graph "
+                      "(kernels back to back, programmatic dependent launch between them)",
             "parallelism": f"replicas x{world} (no data-path collective)",
         },
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": pk["hbm_gbs"],

@@ -126,29 +126,23 @@ awq_status launch_tc_bn(const __half* Xop, int64_t M, const void* Aop, int64_t a
   return launch_tc<256, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
 }
 
-// Streaming decode GEMM (M <= 16, 4-bit): returns AWQ_ERR_UNSUPPORTED when the shape does
-// not suit it (the caller then uses the register-streaming kernel).
+// Streaming decode GEMM (M <= 16, 4-bit), launched with programmatic dependent launch.
+// Returns AWQ_ERR_UNSUPPORTED when the shape does not suit it (X does not fit in shared
+// memory, or N is not a multiple of 16); the caller then uses the register-streaming kernel.
 constexpr int kSmemLimit = 232448;   // 227 KB per CTA on sm_100
 
-template <int kNTiles>
+template <int kNTiles, bool kOffset>
 awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweight,
                               const __half* scales, const uint8_t* zeros, int64_t N, int64_t K,
                               const float* inv_s, __half* y, cudaStream_t st) {
-  if (N % 16 != 0) return AWQ_ERR_UNSUPPORTED;
-  awq::G2Smem lay;
-  lay.x_bytes = static_cast<int>(round_up(M * K * 2, 128));
-  int slots = 8;
-  while (slots >= 2) {
-    lay.slots = slots;
-    if (lay.template total<kNTiles>() <= kSmemLimit) break;
-    slots /= 2;
-  }
-  if (slots < 2) return AWQ_ERR_UNSUPPORTED;
-  const int smem = lay.template total<kNTiles>();
+  if (N % 16 != 0 || K / awq::kGroup > 65535) return AWQ_ERR_UNSUPPORTED;
+  const awq::G4Smem lay = awq::G4Smem::make(static_cast<int>(M), K, kNTiles);
+  const int smem = lay.total(kNTiles);
+  if (smem > kSmemLimit) return AWQ_ERR_UNSUPPORTED;
   static bool attr_set[kMaxDevices] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
-  auto kern = awq::gemv_stream_kernel<kNTiles>;
+  auto kern = awq::gemv_stream_kernel<kNTiles, kOffset>;
   if (!attr_set[dev]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
         cudaSuccess)
@@ -156,7 +150,7 @@ awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweigh
     attr_set[dev] = true;
   }
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, awq::kG2Threads, smem) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, awq::kG4Threads, smem) !=
           cudaSuccess ||
       per_sm < 1)
     return AWQ_ERR_CUDA;
@@ -164,16 +158,16 @@ awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweigh
   const int64_t resident = static_cast<int64_t>(num_sms()) * per_sm;
   const unsigned grid = static_cast<unsigned>(tiles < resident ? tiles : resident);
   CUtensorMap tw, ts, tz;
-  if (!make_tmap_2d(&tw, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, 16, awq::kG2KC / 8,
-                    false) ||
+  if (!make_tmap_2d(&tw, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, 16,
+                    awq::kG4KC / 8, false) ||
       !make_tmap_2d(&ts, scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K / awq::kGroup, N,
-                    awq::kG2Warps, 16, false) ||
+                    awq::kG4Groups, 16, false) ||
       !make_tmap_2d(&tz, zeros, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / awq::kGroup, N,
-                    awq::kG2Warps, 16, false))
+                    awq::kG4Groups, 16, false))
     return AWQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(awq::kG2Threads);
+  cfg.blockDim = dim3(awq::kG4Threads);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -182,7 +176,8 @@ awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweigh
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int m32 = static_cast<int>(M);
-  if (cudaLaunchKernelEx(&cfg, kern, tw, ts, tz, qweight, x, m32, N, K, inv_s, y, lay) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kern, tw, ts, tz, qweight, x, m32, N, K, inv_s, y, lay) !=
+      cudaSuccess)
     return AWQ_ERR_CUDA;
   return launch_status();
 }
@@ -391,8 +386,10 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
   __half* y = reinterpret_cast<__half*>(Y);
 
   if (M <= 16 && bits == 4) {
-    awq_status r = M <= 8 ? launch_gemv_stream<1>(x, M, qweight, sc, zeros, N, K, inv_s, y, st)
-                          : launch_gemv_stream<2>(x, M, qweight, sc, zeros, N, K, inv_s, y, st);
+    awq_status r =
+        M == 1  ? launch_gemv_stream<1, true>(x, M, qweight, sc, zeros, N, K, inv_s, y, st)
+        : M <= 8 ? launch_gemv_stream<1, false>(x, M, qweight, sc, zeros, N, K, inv_s, y, st)
+                 : launch_gemv_stream<2, false>(x, M, qweight, sc, zeros, N, K, inv_s, y, st);
     if (r != AWQ_ERR_UNSUPPORTED) return r;
     const unsigned grid = static_cast<unsigned>((N + awq::kGemvRows - 1) / awq::kGemvRows);
     if (M <= 8)

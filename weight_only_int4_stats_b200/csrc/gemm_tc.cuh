@@ -87,18 +87,20 @@ __device__ __forceinline__ uint4 dequant_word_scaled(uint32_t w, __half2 bias_lo
 }
 
 // 3-bit: the fp16 pair (q - z) * sc for k-offsets (2e, 2e+1) of chunk i (k = 8i..8i+7) of a
-// 32-k block whose low-bit words are w0 (offsets 0..15) / w1 (16..31) and whose bit-2 word,
-// pre-shifted left by 2, is w2s.
+// 32-k block whose low-bit words are w0 (offsets 0..15) / w1 (16..31) and whose bit-2 word
+// is w2 (the pair's two bits sit at bits hb and hb + 16; both are moved to bit 2 of their
+// 16-bit half by a single shift whose direction is fixed at compile time).
 template <int kI, int kE>
-__device__ __forceinline__ uint32_t dequant3_pair(uint32_t w0, uint32_t w1, uint32_t w2s,
+__device__ __forceinline__ uint32_t dequant3_pair(uint32_t w0, uint32_t w1, uint32_t w2,
                                                   __half2 bias_lo, __half2 sc2) {
   constexpr int pp = 4 * (kI & 1) + kE;     // 2-bit field of the pair inside its low word
   constexpr int hb = 4 * kI + kE;           // bit of the pair inside the bit-2 word
   const uint32_t wlo = (kI < 2) ? w0 : w1;
   const uint32_t lo = lop3_and_or(wlo >> (2 * pp), 0x00030003u, 0x64006400u);
+  const uint32_t hs = hb >= 2 ? (w2 >> (hb >= 2 ? hb - 2 : 0)) : (w2 << (hb < 2 ? 2 - hb : 0));
   uint32_t v;
-  // (w2s >> hb) & 0x00040004 | lo
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(v) : "r"(w2s >> hb), "r"(0x00040004u), "r"(lo));
+  // (hs & 0x00040004) | lo
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(v) : "r"(hs), "r"(0x00040004u), "r"(lo));
   return h2_as_u32(__hmul2(__hsub2(u32_as_h2(v), bias_lo), sc2));
 }
 
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         } else {
           const uint32_t* pw = reinterpret_cast<const uint32_t*>(
               smem + L::kPOff + ps * L::kPBytes + r * 48 + 12 * (2 * (kb & 1) + h));
-          const uint32_t w0 = pw[0], w1 = pw[1], w2s = pw[2] << 2;
+          const uint32_t w0 = pw[0], w1 = pw[1], w2s = pw[2];
           uint4 o;
 #define AWQ_DQ3_CHUNK(I)                                                   \
   o.x = dequant3_pair<I, 0>(w0, w1, w2s, lo, sc);                         \

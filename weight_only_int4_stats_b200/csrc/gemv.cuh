@@ -193,87 +193,116 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_w4a16_kernel(
 namespace awq {
 
 // ---------------------------------------------------------------------------------------
-// Streaming decode GEMM (the default decode path).
+// Streaming decode GEMM (the default decode path for M <= 16 when X fits in shared memory).
 //
-// Each CTA owns a contiguous range of whole 16-row tiles, so no output is split across CTAs
-// and the result does not depend on the grid. One producer thread walks the CTA's
-// (tile, 1024-k chunk) units and streams each unit's packed weights ([16 rows, 128 words]),
-// fp16 scales and uint8 zeros ([8 groups, 16 rows] each) with TMA into an 8-slot shared
-// memory ring. Under programmatic dependent launch the kernel starts while the previous
-// kernel on the stream is still finishing: before griddepcontrol.wait it only issues L2
-// prefetches of its weights, scales and zeros (coherent with any write of that kernel, so
-// even a quantize-and-pack directly before it is safe), and every shared-memory load comes
-// after the wait and hits L2. X ([M, K], small at decode) is bulk-copied into shared memory
-// once, after the wait. Eight consumer warps
-// each take one 128-wide group of every unit (the register-only dequant + mma.sync of the
-// kernel above, fed from shared memory) and keep per-tile fp32 sums; at the end of a tile
-// the eight warps' sums are added in a fixed order and written as fp16.
+// Persistent: the grid is sized to the resident capacity and CTA b owns the contiguous
+// range of whole 16-row tiles [b*T/P, (b+1)*T/P), so no output is split across CTAs and the
+// result does not depend on the grid. One producer thread walks the CTA's (tile, 2048-k
+// chunk) units and streams each unit's packed weights ([16 rows, 256 words] = 16 KB), fp16
+// scales and uint8 zeros ([16 groups, 16 rows]) with TMA into a 4-slot shared-memory ring.
+//
+// Programmatic dependent launch: the kernel may start while the previous kernel on the
+// stream is still running. Before griddepcontrol.wait the producer only issues L2 bulk
+// prefetches of the CTA's weight rows (coherent with any write of that kernel, so even a
+// quantize-and-pack just before it is safe); every shared-memory load comes after the wait.
+// X ([M, K], small at decode) is then bulk-copied into shared memory once per CTA.
+//
+// Eight consumer warps each take two 128-wide groups of every unit (two independent MMA
+// chains) with register-only dequantization feeding mma.sync m16n8k16 (weights as the
+// 16-row A operand, activations as the 8-column B operand). Two dequantization forms:
+//  * M = 1 (kOffset): a mask-and-or with 0x6400 turns the nibble pair (k0, k1) of a word
+//    into the exact fp16 values (1024 + q0, 1024 + q1) and the pair (k2, k3), stored 4 bits
+//    higher, into (1024 + 16 q2, 1024 + 16 q3) (the same after a shift by 8 for k4..k7);
+//    these go to the MMA unchanged against X staged with columns k%8 in {2,3,6,7} divided by
+//    16 (exact in fp16), so per group the MMA returns sum_k x_k q_k + C1 with
+//    C1 = 1024 * sum_k xs_k; with C2 = sum_k x_k the group adds s * (mma - C1 - z C2).
+//    C1 and C2 are computed once per CTA. Five integer operations per packed word; the fp32
+//    cancellation of the 1024 offset keeps about 13 significant bits of each group sum.
+//  * M > 1: one fp16 subtract (or multiply-add) per pair leaves the exact q - z first.
+// Per-tile sums of the eight warps are added in a fixed order and stored as fp16.
 // ---------------------------------------------------------------------------------------
-constexpr int kG2Warps = 8;                       // consumer warps = groups per unit
-constexpr int kG2Threads = (kG2Warps + 1) * 32;   // + one producer warp
-constexpr int kG2KC = kG2Warps * kGroup;          // k per unit (1024)
-constexpr int kG2WBytes = kGemvRows * (kG2KC / 2);          // 8192: packed weights
-constexpr int kG2SBytes = kG2Warps * kGemvRows * 2;         // 256: fp16 scales
-constexpr int kG2ZBytes = kG2Warps * kGemvRows;             // 128: uint8 zeros
-constexpr int kG2SlotBytes = kG2WBytes + kG2SBytes + kG2ZBytes;   // 8576 (multiple of 128)
+constexpr int kG4Warps = 8;                        // consumer warps
+constexpr int kG4Threads = (kG4Warps + 1) * 32;    // + one producer warp
+constexpr int kG4Groups = 2 * kG4Warps;            // groups per unit
+constexpr int kG4KC = kG4Groups * kGroup;          // k per unit (2048)
+constexpr int kG4WBytes = kGemvRows * (kG4KC / 2);             // 16384
+constexpr int kG4SBytes = kG4Groups * kGemvRows * 2;           // 512
+constexpr int kG4ZBytes = kG4Groups * kGemvRows;               // 256
+constexpr int kG4SlotBytes = kG4WBytes + kG4SBytes + kG4ZBytes; // 17152 (multiple of 128)
+constexpr int kG4Slots = 4;
 
-struct G2Smem {
-  int x_bytes;      // M * K * 2 rounded up to 128
-  int slots;
-  __host__ __device__ int slot_off() const { return x_bytes; }
-  __host__ __device__ int bar_off() const { return x_bytes + slots * kG2SlotBytes; }
-  template <int kNTiles>
-  __host__ __device__ int red_off() const { return bar_off() + (2 * slots + 1) * 8 + 8; }
-  template <int kNTiles>
-  __host__ __device__ int total() const {
-    return red_off<kNTiles>() + kG2Warps * kNTiles * 4 * 32 * 4;
+struct G4Smem {
+  int x_bytes;   // M * K * 2, rounded up to 128
+  int c_bytes;   // C1/C2 per (group, token)
+  __host__ __device__ int c_off() const { return x_bytes; }
+  __host__ __device__ int slot_off() const { return x_bytes + c_bytes; }
+  __host__ __device__ int bar_off() const { return slot_off() + kG4Slots * kG4SlotBytes; }
+  __host__ __device__ int red_off() const { return bar_off() + (2 * kG4Slots + 2) * 8; }
+  __host__ __device__ int total(int n_tiles) const {
+    return red_off() + kG4Warps * n_tiles * 4 * 32 * 4;
+  }
+  __host__ __device__ static G4Smem make(int M, int64_t K, int n_tiles) {
+    G4Smem l;
+    l.x_bytes = static_cast<int>((static_cast<int64_t>(M) * K * 2 + 127) / 128 * 128);
+    l.c_bytes = static_cast<int>(((K / kGroup) * 8 * n_tiles * 2 * 4 + 127) / 128 * 128);
+    return l;
   }
 };
 
-template <int kNTiles>
-__global__ void __launch_bounds__(kG2Threads) gemv_stream_kernel(
+// One packed word -> the raw fp16 pairs (1024+q0,1024+q1), (1024+16q2,1024+16q3),
+// (1024+q4,1024+q5), (1024+16q6,1024+16q7).
+__device__ __forceinline__ void raw_word(uint32_t w, uint32_t (&v)[4]) {
+  const uint32_t w8 = w >> 8;
+  v[0] = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
+  v[1] = lop3_and_or(w, 0x00F000F0u, 0x64006400u);
+  v[2] = lop3_and_or(w8, 0x000F000Fu, 0x64006400u);
+  v[3] = lop3_and_or(w8, 0x00F000F0u, 0x64006400u);
+}
+
+template <int kNTiles, bool kOffset>
+__global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
     const __grid_constant__ CUtensorMap tmap_z, const uint32_t* __restrict__ qweight,
     const __half* __restrict__ X, int M, int64_t N, int64_t K, const float* __restrict__ inv_s,
-    __half* __restrict__ Y, G2Smem lay) {
+    __half* __restrict__ Y, G4Smem lay) {
   extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int kTok = 8 * kNTiles;
   __half* xs = reinterpret_cast<__half*>(smem);
+  float* cc = reinterpret_cast<float*>(smem + lay.c_off());
   uint8_t* slots = smem + lay.slot_off();
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bar_off());
-  uint64_t* empty = full + lay.slots;
-  uint64_t* xfull = empty + lay.slots;
-  float* red = reinterpret_cast<float*>(smem + lay.template red_off<kNTiles>());
+  uint64_t* empty = full + kG4Slots;
+  uint64_t* xfull = empty + kG4Slots;
+  float* red = reinterpret_cast<float*>(smem + lay.red_off());
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t T = (N + kGemvRows - 1) / kGemvRows;
   const int64_t P = gridDim.x;
   const int64_t t0 = blockIdx.x * T / P, t1 = (blockIdx.x + 1) * T / P;
-  const int64_t C = (K + kG2KC - 1) / kG2KC;
+  const int Ki = static_cast<int>(K);
+  const int G = Ki / kGroup;
+  const int C = (Ki + kG4KC - 1) / kG4KC;
   const int64_t units = (t1 - t0) * C;
-  const int64_t G = K / kGroup;
-  const int S = lay.slots;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) {
+    for (int i = 0; i < kG4Slots; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kG2Warps);
+      mbar_init(&empty[i], kG4Warps);
     }
     mbar_init(xfull, 1);
     fence_barrier_init();
   }
   __syncthreads();
 
-  if (warp == kG2Warps) {
+  if (warp == kG4Warps) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       pdl_launch_dependents();
       tma_prefetch_desc(&tmap_w);
       tma_prefetch_desc(&tmap_s);
       tma_prefetch_desc(&tmap_z);
-      // HBM -> L2 for everything this CTA will read: its rows of packed weights are one
-      // contiguous range; scales and zeros are fetched per unit through their tensor maps.
-      {
+      {   // HBM -> L2 for this CTA's weight rows (one contiguous range)
         const int64_t row_bytes = K / 2;
         const int64_t r0 = t0 * kGemvRows, r1 = t1 * kGemvRows < N ? t1 * kGemvRows : N;
         const uint8_t* wrow = reinterpret_cast<const uint8_t*>(qweight) + r0 * row_bytes;
@@ -281,55 +310,89 @@ __global__ void __launch_bounds__(kG2Threads) gemv_stream_kernel(
         for (int64_t off = 0; off < bytes; off += 65536)
           prefetch_l2_bulk(wrow + off, static_cast<uint32_t>(bytes - off < 65536 ? bytes - off : 65536));
       }
-      for (int64_t u = 0; u < units; ++u) {
-        const int64_t tile = t0 + u / C, chunk = u % C;
-        prefetch_l2_tile_2d(&tmap_s, static_cast<int32_t>(tile * kGemvRows),
-                            static_cast<int32_t>(chunk * kG2Warps));
-        prefetch_l2_tile_2d(&tmap_z, static_cast<int32_t>(tile * kGemvRows),
-                            static_cast<int32_t>(chunk * kG2Warps));
-      }
       pdl_wait();
       mbar_arrive_expect_tx(xfull, static_cast<uint32_t>(M * K * 2));
       bulk_load_1d(xs, X, static_cast<uint32_t>(M * K * 2), xfull);
+      int slot = 0, chunk = 0;
+      uint32_t ph = 0;
+      int64_t tile = t0;
       for (int64_t u = 0; u < units; ++u) {
-        const int slot = static_cast<int>(u % S);
-        const uint32_t ph = static_cast<uint32_t>((u / S) & 1);
         if (!mbar_wait(&empty[slot], ph ^ 1)) break;
-        const int64_t tile = t0 + u / C, chunk = u % C;
-        uint8_t* sb = slots + slot * kG2SlotBytes;
-        mbar_arrive_expect_tx(&full[slot], kG2SlotBytes);
-        tma_load_2d(sb, &tmap_w, &full[slot], static_cast<int32_t>(chunk * (kG2KC / 8)),
-                    static_cast<int32_t>(tile * kGemvRows));
-        tma_load_2d(sb + kG2WBytes, &tmap_s, &full[slot], static_cast<int32_t>(tile * kGemvRows),
-                    static_cast<int32_t>(chunk * kG2Warps));
-        tma_load_2d(sb + kG2WBytes + kG2SBytes, &tmap_z, &full[slot],
-                    static_cast<int32_t>(tile * kGemvRows), static_cast<int32_t>(chunk * kG2Warps));
+        uint8_t* sb = slots + slot * kG4SlotBytes;
+        mbar_arrive_expect_tx(&full[slot], kG4SlotBytes);
+        const int32_t row = static_cast<int32_t>(tile * kGemvRows);
+        tma_load_2d(sb, &tmap_w, &full[slot], chunk * (kG4KC / 8), row);
+        tma_load_2d(sb + kG4WBytes, &tmap_s, &full[slot], row, chunk * kG4Groups);
+        tma_load_2d(sb + kG4WBytes + kG4SBytes, &tmap_z, &full[slot], row, chunk * kG4Groups);
+        if (++slot == kG4Slots) { slot = 0; ph ^= 1; }
+        if (++chunk == C) { chunk = 0; ++tile; }
       }
     }
     return;
   }
 
   // ------------------------------------------------------------------ consumers
+  // A timed-out wait clears `ok`; the warp then skips further waits and arithmetic but still
+  // runs every named barrier, so the consumer warps cannot deadlock one another.
   const int r = lane >> 2, c = lane & 3;
-  // A timed-out wait clears `ok`; the warp then skips all further waits and arithmetic but
-  // still runs every named barrier, so the consumer warps can never deadlock each other.
   bool ok = __all_sync(0xffffffffu, mbar_wait(xfull, 0));
-  if (inv_s != nullptr) {
-    // x <- fp16(x * inv_s), in place, by the 256 consumer threads
-    const int64_t n8 = static_cast<int64_t>(M) * K / 8;
-    for (int64_t i = threadIdx.x; ok && i < n8; i += kG2Warps * 32) {
-      const int64_t k = (i * 8) % K;
+  if (inv_s != nullptr || kOffset) {
+    // x <- fp16(x * inv_s); for kOffset also divide columns k%8 in {2,3,6,7} by 16
+    const int n8 = M * Ki / 8;
+    for (int i = threadIdx.x; ok && i < n8; i += kG4Warps * 32) {
       uint4 v = reinterpret_cast<uint4*>(xs)[i];
-      const float4 s0 = *reinterpret_cast<const float4*>(inv_s + k);
-      const float4 s1 = *reinterpret_cast<const float4*>(inv_s + k + 4);
-      float2 f;
-      f = __half22float2(u32_as_h2(v.x)); v.x = h2_as_u32(__floats2half2_rn(f.x * s0.x, f.y * s0.y));
-      f = __half22float2(u32_as_h2(v.y)); v.y = h2_as_u32(__floats2half2_rn(f.x * s0.z, f.y * s0.w));
-      f = __half22float2(u32_as_h2(v.z)); v.z = h2_as_u32(__floats2half2_rn(f.x * s1.x, f.y * s1.y));
-      f = __half22float2(u32_as_h2(v.w)); v.w = h2_as_u32(__floats2half2_rn(f.x * s1.z, f.y * s1.w));
+      if (inv_s != nullptr) {
+        const int k = (i * 8) % Ki;
+        const float4 s0 = *reinterpret_cast<const float4*>(inv_s + k);
+        const float4 s1 = *reinterpret_cast<const float4*>(inv_s + k + 4);
+        float2 f;
+        f = __half22float2(u32_as_h2(v.x)); v.x = h2_as_u32(__floats2half2_rn(f.x * s0.x, f.y * s0.y));
+        f = __half22float2(u32_as_h2(v.y)); v.y = h2_as_u32(__floats2half2_rn(f.x * s0.z, f.y * s0.w));
+        f = __half22float2(u32_as_h2(v.z)); v.z = h2_as_u32(__floats2half2_rn(f.x * s1.x, f.y * s1.y));
+        f = __half22float2(u32_as_h2(v.w)); v.w = h2_as_u32(__floats2half2_rn(f.x * s1.z, f.y * s1.w));
+      }
+      if (kOffset) {
+        const __half2 sixteenth = __float2half2_rn(0.0625f);
+        v.y = h2_as_u32(__hmul2(u32_as_h2(v.y), sixteenth));
+        v.w = h2_as_u32(__hmul2(u32_as_h2(v.w), sixteenth));
+      }
       reinterpret_cast<uint4*>(xs)[i] = v;
     }
-    named_bar_sync(1, kG2Warps * 32);
+    named_bar_sync(1, kG4Warps * 32);
+  }
+  if (kOffset) {
+    // C1 = 1024 * sum(xs), C2 = sum(x) per (group, token < M); tokens >= M get zeros.
+    // 8 threads per (group, token) pair, 4 pairs per warp and pass, three xor-shuffles.
+    const int sub = lane & 7;
+    const int npairs = G * M;
+    for (int base = warp * 4; base < npairs; base += kG4Warps * 4) {
+      const int pr = base + (lane >> 3);
+      const bool live = ok && pr < npairs;
+      const int g = live ? pr / M : 0, m = live ? pr % M : 0;
+      const uint4* src = reinterpret_cast<const uint4*>(xs + m * Ki + g * kGroup + 16 * sub);
+      float c1 = 0.0f, c2 = 0.0f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint4 u = src[h];
+        const float2 lx = __half22float2(u32_as_h2(u.x)), hy = __half22float2(u32_as_h2(u.y));
+        const float2 lz = __half22float2(u32_as_h2(u.z)), hw = __half22float2(u32_as_h2(u.w));
+        const float lo = (lx.x + lx.y) + (lz.x + lz.y), hi = (hy.x + hy.y) + (hw.x + hw.y);
+        c1 += lo + hi;
+        c2 += lo + 16.0f * hi;
+      }
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        c1 += __shfl_xor_sync(0xffffffffu, c1, o);
+        c2 += __shfl_xor_sync(0xffffffffu, c2, o);
+      }
+      if (sub == 0 && live) {
+        cc[(g * kTok + m) * 2] = 1024.0f * c1;
+        cc[(g * kTok + m) * 2 + 1] = c2;
+      }
+    }
+    for (int i = threadIdx.x; i < G * kTok; i += kG4Warps * 32)
+      if (i % kTok >= M) { cc[2 * i] = 0.0f; cc[2 * i + 1] = 0.0f; }
+    named_bar_sync(1, kG4Warps * 32);
   }
 
   float total[kNTiles][4];
@@ -338,59 +401,83 @@ __global__ void __launch_bounds__(kG2Threads) gemv_stream_kernel(
 #pragma unroll
     for (int i = 0; i < 4; ++i) total[t][i] = 0.0f;
 
+  int slot = 0, chunk = 0;
+  uint32_t ph = 0;
+  int64_t tile = t0;
   for (int64_t u = 0; u < units; ++u) {
-    const int slot = static_cast<int>(u % S);
-    const uint32_t ph = static_cast<uint32_t>((u / S) & 1);
     ok = __all_sync(0xffffffffu, ok && mbar_wait(&full[slot], ph));
-    const int64_t tile = t0 + u / C, chunk = u % C;
-    const int64_t g = chunk * kG2Warps + warp;
-    const uint8_t* sb = slots + slot * kG2SlotBytes;
-    if (ok && g < G) {
-      const uint4 wA = *reinterpret_cast<const uint4*>(sb + r * (kG2KC / 2) + (warp * 16 + 4 * c) * 4);
-      const uint4 wB =
-          *reinterpret_cast<const uint4*>(sb + (r + 8) * (kG2KC / 2) + (warp * 16 + 4 * c) * 4);
-      const __half* ss = reinterpret_cast<const __half*>(sb + kG2WBytes) + warp * kGemvRows;
-      const uint8_t* zz = sb + kG2WBytes + kG2SBytes + warp * kGemvRows;
-      const uint32_t zA = zz[r], zB = zz[r + 8];
-      const float scA = __half2float(ss[r]), scB = __half2float(ss[r + 8]);
-      const __half2 loA = u32_as_h2((0x6400u | zA) * 0x00010001u);
-      const __half2 hiA = __hneg2(u32_as_h2((0x5400u | (zA << 4)) * 0x00010001u));
-      const __half2 loB = u32_as_h2((0x6400u | zB) * 0x00010001u);
-      const __half2 hiB = __hneg2(u32_as_h2((0x5400u | (zB << 4)) * 0x00010001u));
-      float acc[kNTiles][4];
+    const uint8_t* sb = slots + slot * kG4SlotBytes;
 #pragma unroll
-      for (int t = 0; t < kNTiles; ++t)
+    for (int q = 0; q < 2; ++q) {
+      const int gl = 2 * warp + q;               // group inside the unit
+      const int g = chunk * kG4Groups + gl;
+      if (ok && g < G) {
+        const uint8_t* wrow = sb + (gl * 16 + 4 * c) * 4;
+        const uint4 wA = *reinterpret_cast<const uint4*>(wrow + r * (kG4KC / 2));
+        const uint4 wB = *reinterpret_cast<const uint4*>(wrow + (r + 8) * (kG4KC / 2));
+        const __half* ss = reinterpret_cast<const __half*>(sb + kG4WBytes) + gl * kGemvRows;
+        const uint8_t* zz = sb + kG4WBytes + kG4SBytes + gl * kGemvRows;
+        const uint32_t zAi = zz[r], zBi = zz[r + 8];
+        const float scA = __half2float(ss[r]), scB = __half2float(ss[r + 8]);
+        float acc[kNTiles][2][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
-      const uint32_t wordsA[4] = {wA.x, wA.y, wA.z, wA.w};
-      const uint32_t wordsB[4] = {wB.x, wB.y, wB.z, wB.w};
-      const int64_t kx = g * kGroup + 32 * c;
+        for (int t = 0; t < kNTiles; ++t)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t qa[4], qb[4];
-        dequant_word_qz(wordsA[j], loA, hiA, qa);
-        dequant_word_qz(wordsB[j], loB, hiB, qb);
+          for (int i = 0; i < 4; ++i) acc[t][0][i] = acc[t][1][i] = 0.0f;
+        const uint32_t wordsA[4] = {wA.x, wA.y, wA.z, wA.w};
+        const uint32_t wordsB[4] = {wB.x, wB.y, wB.z, wB.w};
+        const int kx = g * kGroup + 32 * c;
+        __half2 loA, hiA, loB, hiB;
+        if (!kOffset) {
+          loA = u32_as_h2((0x6400u | zAi) * 0x00010001u);
+          hiA = u32_as_h2((0xD400u | (zAi << 4)) * 0x00010001u);
+          loB = u32_as_h2((0x6400u | zBi) * 0x00010001u);
+          hiB = u32_as_h2((0xD400u | (zBi << 4)) * 0x00010001u);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t va[4], vb[4];
+          if (kOffset) {
+            raw_word(wordsA[j], va);
+            raw_word(wordsB[j], vb);
+          } else {
+            dequant_word_qz(wordsA[j], loA, hiA, va);
+            dequant_word_qz(wordsB[j], loB, hiB, vb);
+          }
+#pragma unroll
+          for (int t = 0; t < kNTiles; ++t) {
+            const int m = r + 8 * t;
+            uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+            if (m < M) xv = *reinterpret_cast<const uint4*>(xs + m * Ki + kx + 8 * j);
+            const uint32_t a0[4] = {va[0], vb[0], va[1], vb[1]};
+            mma_16816(acc[t][j & 1], a0, xv.x, xv.y);
+            const uint32_t a1[4] = {va[2], vb[2], va[3], vb[3]};
+            mma_16816(acc[t][j & 1], a1, xv.z, xv.w);
+          }
+        }
 #pragma unroll
         for (int t = 0; t < kNTiles; ++t) {
-          const int m = r + 8 * t;
-          uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-          if (m < M) xv = *reinterpret_cast<const uint4*>(xs + m * K + kx + 8 * j);
-          const uint32_t a0[4] = {qa[0], qb[0], qa[1], qb[1]};
-          mma_16816(acc[t], a0, xv.x, xv.y);
-          const uint32_t a1[4] = {qa[2], qb[2], qa[3], qb[3]};
-          mma_16816(acc[t], a1, xv.z, xv.w);
-        }
-      }
+          float d[4];
 #pragma unroll
-      for (int t = 0; t < kNTiles; ++t) {
-        total[t][0] = fmaf(scA, acc[t][0], total[t][0]);
-        total[t][1] = fmaf(scA, acc[t][1], total[t][1]);
-        total[t][2] = fmaf(scB, acc[t][2], total[t][2]);
-        total[t][3] = fmaf(scB, acc[t][3], total[t][3]);
+          for (int i = 0; i < 4; ++i) d[i] = acc[t][0][i] + acc[t][1][i];
+          if (kOffset) {
+            const float zA = static_cast<float>(zAi), zB = static_cast<float>(zBi);
+            const float4 cm = *reinterpret_cast<const float4*>(cc + (g * kTok + 8 * t + 2 * c) * 2);
+            d[0] -= fmaf(zA, cm.y, cm.x);
+            d[1] -= fmaf(zA, cm.w, cm.z);
+            d[2] -= fmaf(zB, cm.y, cm.x);
+            d[3] -= fmaf(zB, cm.w, cm.z);
+          }
+          total[t][0] = fmaf(scA, d[0], total[t][0]);
+          total[t][1] = fmaf(scA, d[1], total[t][1]);
+          total[t][2] = fmaf(scB, d[2], total[t][2]);
+          total[t][3] = fmaf(scB, d[3], total[t][3]);
+        }
       }
     }
     __syncwarp();
     if (ok && lane == 0) mbar_arrive(&empty[slot]);
+    if (++slot == kG4Slots) { slot = 0; ph ^= 1; }
 
     if (chunk == C - 1) {
       // tile complete: fixed-order sum over the eight consumer warps, fp16 store
@@ -401,16 +488,16 @@ __global__ void __launch_bounds__(kG2Threads) gemv_stream_kernel(
           red[((warp * kNTiles + t) * 4 + i) * 32 + lane] = total[t][i];
           total[t][i] = 0.0f;
         }
-      named_bar_sync(1, kG2Warps * 32);
+      named_bar_sync(1, kG4Warps * 32);
       if (ok && warp < kNTiles) {
         const int t = warp;
         float v[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          float s = 0.0f;
+          float sum = 0.0f;
 #pragma unroll
-          for (int w = 0; w < kG2Warps; ++w) s += red[((w * kNTiles + t) * 4 + i) * 32 + lane];
-          v[i] = s;
+          for (int w = 0; w < kG4Warps; ++w) sum += red[((w * kNTiles + t) * 4 + i) * 32 + lane];
+          v[i] = sum;
         }
         const int64_t nA = tile * kGemvRows + r, nB = nA + 8;
         const int m0 = 8 * t + 2 * c, m1 = m0 + 1;
@@ -423,8 +510,9 @@ __global__ void __launch_bounds__(kG2Threads) gemv_stream_kernel(
           if (m1 < M) Y[static_cast<int64_t>(m1) * N + nB] = __float2half_rn(v[3]);
         }
       }
-      named_bar_sync(1, kG2Warps * 32);
+      named_bar_sync(1, kG4Warps * 32);
     }
+    if (++chunk == C) { chunk = 0; ++tile; }
   }
 }
 
