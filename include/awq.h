@@ -87,6 +87,26 @@ AWQ_API size_t awq_act_stats_workspace_size(int64_t M, int64_t K);
 AWQ_API awq_status awq_act_stats(const awq_f16* X, int64_t M, int64_t K, float* s_x, void* workspace,
                          size_t ws_bytes, void* stream);
 
+/* Same result as awq_act_stats, for callers that cannot allocate device memory. The AWQ
+ * pages have no counterpart to this call; it exists because some callers have no way to
+ * provide a workspace: a plugin inside another framework's engine that is handed only its
+ * input and output pointers, or a latency-critical path that must not call cudaMalloc
+ * (which can synchronize the whole device).
+ * Instead of a workspace it uses one 4 MiB array of device memory that the library defines
+ * at file scope; every GPU that loads the library holds that array until the process exits.
+ * Limits: K <= 65536 (K a multiple of 8, M >= 1); a larger K returns AWQ_ERR_INVALID_ARG
+ * before anything is launched. The row split is capped so the partial sums fit the array,
+ * which can change the fp64 summation order relative to awq_act_stats (the results agree
+ * whenever those sums are exact, as they are for fp16 inputs of moderate range).
+ * The first call on each device looks up the array's device address (with that device
+ * current) and caches it; make that first call before any stream capture.
+ * Every call shares the one array: calls that may overlap on the GPU (different streams,
+ * or different host threads on the same device) race on it and must be serialized by the
+ * caller. Nothing in the array needs clearing between calls: each call overwrites every
+ * partial sum it reads. No device memory is allocated or freed by this call. */
+AWQ_API awq_status awq_act_stats_noalloc(const awq_f16* X, int64_t M, int64_t K, float* s_x,
+                                         void* stream);
+
 /* ---------------------------------------------------------------- quantize and pack
  * robotsatlas.com "AWQ", "Components: Group-wise 4-bit quantization" and "Hyperparameters";
  * builderai.tools "AWQ", "About" ("writes real INT4 weights"). Quantizes W diag(s) per

@@ -14,7 +14,7 @@ import torch
 
 __all__ = [
     "AwqError", "lib", "library_path", "GROUP",
-    "awq_act_stats", "awq_quantize_pack", "awq_search_scale", "awq_gemm_w4a16",
+    "awq_act_stats", "awq_act_stats_noalloc", "awq_quantize_pack", "awq_search_scale", "awq_gemm_w4a16",
     "awq_check_error", "packed_words_per_row",
 ]
 
@@ -52,6 +52,7 @@ def lib() -> ctypes.CDLL:
             "awq_check_error": (I32, [P]),
             "awq_act_stats_workspace_size": (SZ, [I64, I64]),
             "awq_act_stats": (I32, [P, I64, I64, P, P, SZ, P]),
+            "awq_act_stats_noalloc": (I32, [P, I64, I64, P, P]),
             "awq_quantize_pack": (I32, [P, I64, I64, P, I32, I32, P, P, P, P]),
             "awq_search_scale_workspace_size": (SZ, [I64, I64, I64, I32]),
             "awq_search_scale": (I32, [P, I64, I64, P, I64, P, P, I32, I32, I32, P, P, P, P, P,
@@ -112,6 +113,19 @@ def awq_act_stats(X: torch.Tensor, out: torch.Tensor | None = None, workspace=No
     ws = _workspace(ws_bytes, X.device) if workspace is None else workspace
     _check("awq_act_stats", lib().awq_act_stats(_ptr(X), M, K, _ptr(s_x), _ptr(ws),
                                                 ws.numel() * ws.element_size(), _stream(stream)))
+    return s_x
+
+
+def awq_act_stats_noalloc(X: torch.Tensor, out: torch.Tensor | None = None,
+                          stream=None) -> torch.Tensor:
+    """awq_act_stats without a workspace: the library's own fixed device array holds the
+    partial sums (K <= 65536; calls that overlap on the GPU race on that array)."""
+    _need(X, torch.float16, "X")
+    M, K = X.shape
+    s_x = torch.empty(K, dtype=torch.float32, device=X.device) if out is None else out
+    _need(s_x, torch.float32, "out")
+    _check("awq_act_stats_noalloc",
+           lib().awq_act_stats_noalloc(_ptr(X), M, K, _ptr(s_x), _stream(stream)))
     return s_x
 
 

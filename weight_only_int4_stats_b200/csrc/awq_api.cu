@@ -246,6 +246,64 @@ awq_status awq_act_stats(const awq_f16* X, int64_t M, int64_t K, float* s_x, voi
   return launch_status();
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------------ act_stats without allocation
+// Scratch for awq_act_stats_noalloc: the fp64 partial sums live in this file-scope device
+// array instead of a caller workspace. Every GPU that loads the library holds it until the
+// process exits. In host code the name is only a stand-in for the symbol, so its device
+// address is looked up once per device (with that device current) and cached.
+namespace {
+constexpr int64_t kNoAllocScratchDoubles = int64_t{1} << 19;   // 4 MiB
+constexpr int64_t kNoAllocMaxK = 65536;                       // >= 8 row slices per call
+static __device__ __align__(256) double g_noalloc_scratch[kNoAllocScratchDoubles];
+
+double* g_noalloc_ptr[kMaxDevices] = {nullptr};
+std::mutex g_noalloc_mu;
+
+awq_status noalloc_scratch(double** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return AWQ_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<double*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return AWQ_OK;
+}
+}  // namespace
+
+extern "C" {
+
+awq_status awq_act_stats_noalloc(const awq_f16* X, int64_t M, int64_t K, float* s_x,
+                                 void* stream) {
+  if (bad_dim(M) || bad_dim(K) || M == 0) return AWQ_ERR_INVALID_ARG;
+  if (K == 0) return AWQ_OK;
+  if (K % 8 != 0 || K > kNoAllocMaxK) return AWQ_ERR_INVALID_ARG;
+  if (!X || !s_x || !aligned16(X) || !aligned16(s_x)) return AWQ_ERR_INVALID_ARG;
+  double* part = nullptr;
+  awq_status s = noalloc_scratch(&part);
+  if (s != AWQ_OK) return s;
+  int splits = awq::act_stats_splits(M, K, num_sms());
+  const int64_t cap = kNoAllocScratchDoubles / K;
+  if (splits > cap) splits = static_cast<int>(cap);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Pass 1 writes every (slice, channel) partial it later reads, so nothing of an earlier
+  // call's contents is used and the array needs no clearing.
+  const int64_t rows_per_split = (M + splits - 1) / splits;
+  dim3 g1(static_cast<unsigned>((K + awq::kStatsCols - 1) / awq::kStatsCols),
+          static_cast<unsigned>(splits));
+  awq::act_stats_partial_kernel<<<g1, 256, 0, st>>>(reinterpret_cast<const __half*>(X), M, K,
+                                                   rows_per_split, part);
+  if ((s = launch_status()) != AWQ_OK) return s;
+  awq::act_stats_finish_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(
+      part, splits, M, K, s_x);
+  return launch_status();
+}
+
 // ------------------------------------------------------------------ quantize_pack
 awq_status awq_quantize_pack(const awq_f16* W, int64_t N, int64_t K, const float* s, int bits,
                              int group, uint32_t* qweight, awq_f16* scales, uint8_t* zeros,
