@@ -60,7 +60,7 @@ typedef uint16_t awq_f16; /* IEEE binary16 storage */
 typedef enum {
   AWQ_OK = 0,
   AWQ_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad shape, unsupported bits/group */
-  AWQ_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement */
+  AWQ_ERR_UNSUPPORTED = 2,   /* valid request the library does not implement */
   AWQ_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the size query's answer */
   AWQ_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (e.g. no GPU, launch) */
   AWQ_ERR_TIMEOUT = 5        /* a kernel's bounded wait ran out (see awq_check_error) */
