@@ -224,6 +224,146 @@ def cpu_oracle_sample(shapes, rows=512, repeats=2):
     return total_bytes / total_t / 1e9, total_t, desc
 
 
+# ----------------------------------------------------------------------------- other rows
+
+def time_call(fn, reps, warm=1):
+    """Median device time of `fn` over `reps` calls (CUDA events on the current stream)."""
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) / 1e3)
+    return statistics.median(ts)
+
+
+def decoder_layer_rows(awq, dev, pk):
+    """The other hot-path rows on the 7B-shaped decoder layer and its 65536-token calibration
+    batch: activation statistics, the 20-point searches (q/k/v and gate/up jointly), packing,
+    and the W4A16 GEMM of every linear over the calibration batch -- timed per stage and as
+    one pipeline. Also quantize-and-pack on the largest prefill weight."""
+    rows = {}
+    acts = synth.decoder_layer_activations()
+    Ws = synth.decoder_layer_weights()
+    alphas = torch.from_numpy(np.arange(20, dtype=np.float32) / np.float32(20)).to(dev)
+    Xd = {k: torch.from_numpy(v).to(dev) for k, v in acts.items()}
+    del acts
+    Wd = {k: torch.from_numpy(v).to(dev) for k, v in Ws.items()}
+    del Ws
+
+    # act_stats (HBM-bound: 2MK bytes)
+    out = []
+    for name in ("hidden", "down_in"):
+        X = Xd[name]
+        M, K = X.shape
+        ws = torch.empty(max(awq.lib().awq_act_stats_workspace_size(M, K), 16), dtype=torch.uint8,
+                         device=dev)
+        sx = torch.empty(K, dtype=torch.float32, device=dev)
+        t = time_call(lambda: awq.awq_act_stats(X, out=sx, workspace=ws), 5)
+        gbs = 2 * M * K / t / 1e9
+        out.append({"M": M, "K": K, "us": t * 1e6, "GB/s": gbs, "frac_hbm": gbs / pk["hbm_gbs"]})
+    rows["act_stats"] = out
+
+    # the joint gate/up search at full size (the largest of the layer's four searches)
+    Wgu = torch.cat([Wd["gate_proj"], Wd["up_proj"]]).contiguous()
+    X = Xd["hidden"]
+    sx = awq.awq_act_stats(X)
+    M, K = X.shape
+    Ngu = Wgu.shape[0]
+    ws = torch.empty(awq.lib().awq_search_scale_workspace_size(M, Ngu, K, 20), dtype=torch.uint8,
+                     device=dev)
+    t = time_call(lambda: awq.awq_search_scale(Wgu, X, sx, alphas, 4, workspace=ws), 2)
+    flops = 20 * 2 * M * Ngu * K
+    rows["search_gate_up"] = {"M": M, "N": Ngu, "K": K, "grid": 20, "ms": t * 1e3,
+                              "TFLOP/s": flops / t / 1e12,
+                              "frac_tensor": flops / t / 1e12 / pk["bf16_tflops"]}
+    del ws, Wgu
+    torch.cuda.empty_cache()
+
+    # the whole layer as one pipeline: stats -> 4 searches -> 7 packs -> 7 GEMMs over the batch
+    jobs = [("hidden", ["q_proj", "k_proj", "v_proj"]), ("hidden", ["gate_proj", "up_proj"]),
+            ("o_in", ["o_proj"]), ("down_in", ["down_proj"])]
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    ev[0].record()
+    stats = {name: awq.awq_act_stats(Xd[name]) for name in ("hidden", "o_in", "down_in")}
+    ev[1].record()
+    chosen = {}
+    search_flops = 0
+    for xname, names in jobs:
+        W = torch.cat([Wd[n] for n in names]).contiguous() if len(names) > 1 else Wd[names[0]]
+        _, best, best_s, _ = awq.awq_search_scale(W, Xd[xname], stats[xname], alphas, 4)
+        search_flops += 20 * 2 * Xd[xname].shape[0] * W.shape[0] * W.shape[1]
+        for n in names:
+            chosen[n] = (best, best_s)
+        del W
+    ev[2].record()
+    packed = {n: awq.awq_quantize_pack(Wd[n], chosen[n][1], 4) for n in Wd}
+    ev[3].record()
+    gemm_flops = 0
+    xin = {"q_proj": "hidden", "k_proj": "hidden", "v_proj": "hidden", "gate_proj": "hidden",
+           "up_proj": "hidden", "o_proj": "o_in", "down_proj": "down_in"}
+    for n, (qw, sc, z) in packed.items():
+        N, K = Wd[n].shape
+        inv = (1.0 / chosen[n][1]).contiguous()
+        Y = awq.awq_gemm_w4a16(Xd[xin[n]], qw, sc, z, N, K, 4, inv_s=inv)
+        gemm_flops += 2 * Xd[xin[n]].shape[0] * N * K
+        del Y
+    ev[4].record()
+    torch.cuda.synchronize()
+    st = [ev[i].elapsed_time(ev[i + 1]) / 1e3 for i in range(4)]
+    rows["decoder_layer_pipeline"] = {
+        "tokens": int(Xd["hidden"].shape[0]), "seconds": sum(st),
+        "act_stats_s": st[0], "search_s": st[1], "pack_s": st[2], "gemm_s": st[3],
+        "search_TFLOP/s": search_flops / st[1] / 1e12, "gemm_TFLOP/s": gemm_flops / st[3] / 1e12,
+        "alpha_index": {n: int(chosen[n][0].item()) for n in chosen},
+    }
+    del Xd, Wd, packed, stats, chosen
+    torch.cuda.empty_cache()
+
+    # quantize-and-pack on the largest prefill weight (HBM-bound)
+    N, K = synth.PREFILL_SHAPES[0]
+    W, mag, _ = synth.prefill_layer(N, K, 1)
+    Wt = torch.from_numpy(W).to(dev)
+    del W
+    s = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(dev)
+    out = []
+    for bits in (4, 3):
+        t = time_call(lambda: awq.awq_quantize_pack(Wt, s, bits), 5)
+        b = 2 * N * K + N * K * bits // 8 + 3 * N * (K // GROUP)
+        out.append({"N": N, "K": K, "bits": bits, "us": t * 1e6, "GB/s": b / t / 1e9,
+                    "frac_hbm": b / t / 1e9 / pk["hbm_gbs"]})
+    rows["quantize_pack"] = out
+    del Wt
+    torch.cuda.empty_cache()
+    return rows
+
+
+def profile_rows(awq, dev):
+    """Small cases of the other kernels for detailed profiling (a few GB on the device):
+    act_stats on one 65536 x 4096 calibration input, quantize-and-pack of one
+    [28672, 8192] weight, and the 20-point search of one [4096, 4096] linear over it."""
+    X = torch.from_numpy(synth.decoder_layer_activations(names=("o_in",))["o_in"]).to(dev)
+    sx = awq.awq_act_stats(X)
+    N, K = synth.PREFILL_SHAPES[0]
+    W, mag, _ = synth.prefill_layer(N, K, 1)
+    Wt = torch.from_numpy(W).to(dev)
+    del W
+    s = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(dev)
+    awq.awq_quantize_pack(Wt, s, 4)
+    del Wt
+    Wo = torch.from_numpy(synth.decoder_layer_weights()["o_proj"]).to(dev)
+    alphas = torch.from_numpy(np.arange(20, dtype=np.float32) / np.float32(20)).to(dev)
+    awq.awq_search_scale(Wo, X, sx, alphas, 4)
+    torch.cuda.synchronize()
+
+
 # ----------------------------------------------------------------------------- main arms
 
 def run_reference(args, world, rank):
@@ -277,6 +417,14 @@ def run_b200(args, world, rank, local):
     l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024)
     pk = peaks()
     stream = torch.cuda.Stream()
+    if args.only == "profile":
+        profile_rows(awq, dev)
+        return
+    if args.only == "rows":
+        rows = decoder_layer_rows(awq, dev, pk)
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "rows": rows}), flush=True)
+        return
 
     # ---- headline: decode GEMM at M = 1 over the three shapes
     shapes = [DecodeShape(awq, N, K, 16, l2, dev) for (N, K) in synth.DECODE_SHAPES]
@@ -366,6 +514,8 @@ def run_b200(args, world, rank, local):
     pf_time = sum(p["ms"] for p in pf4) / 1e3
     pf_value = pf_flops / pf_time / 1e12 if pf4 else None
 
+    rows = decoder_layer_rows(awq, dev, pk) if args.only == "all" else None
+
     if rank != 0:
         return
     cpu_gbs, cpu_t, cpu_desc = (cpu_oracle_sample(synth.DECODE_SHAPES) if args.only == "all"
@@ -392,6 +542,7 @@ def run_b200(args, world, rank, local):
                     "frac": pf_value / pk["bf16_tflops"] if prefill else None,
                     "kernel": "tc_gemm_kernel"},
         "sweep": sweep,
+        "rows": rows,
         "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": cpu_desc, "seconds": cpu_t},
         "e2e": e2e,
@@ -407,7 +558,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--only", choices=["all", "decode", "prefill"], default="all",
+    ap.add_argument("--only", choices=["all", "decode", "prefill", "rows", "profile"],
+                    default="all",
                     help="run one section only (used by the profiling commands)")
     args = ap.parse_args()
     if args.warmup < 3:

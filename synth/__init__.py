@@ -153,16 +153,19 @@ def decoder_layer_weights(hidden: int = 4096, mlp: int = 11008):
     return {name: random_weight(rng, *shapes[name], 0.02) for name, _, _ in _DECODER_LINEARS}
 
 
-def decoder_layer_activations(tokens: int = 128 * 512, hidden: int = 4096, mlp: int = 11008):
-    """Seed 4 (separate stream from the weights): three calibration inputs of ``tokens`` rows,
-    each N(0, 1) times its own lognormal(0, 0.7) channel magnitudes with round(0.01 K)
-    outlier channels multiplied by U(10, 50): the hidden state X (input of q/k/v and
-    gate/up), X_o (input of o_proj) and X_d (input of down_proj), drawn in that order.
-    A smaller ``tokens`` gives the leading rows of the same stream only when ``tokens``
-    is a multiple of the draw chunk; callers that compare runs use the same ``tokens``."""
-    rng = _rng(4, tokens, hidden, mlp)
+def decoder_layer_activations(tokens: int = 128 * 512, hidden: int = 4096, mlp: int = 11008,
+                              names=("hidden", "o_in", "down_in")):
+    """Seed 4: the layer's three calibration inputs of ``tokens`` rows, each N(0, 1) times its
+    own lognormal(0, 0.7) channel magnitudes with round(0.01 K) outlier channels multiplied
+    by U(10, 50): the hidden state X (input of q/k/v and gate/up), X_o (input of o_proj) and
+    X_d (input of down_proj). Each input has its own stream (SeedSequence [4, tokens, K, i],
+    i = 0, 1, 2 in that order), drawing magnitudes, outlier indices, gains, then X, so any
+    subset can be generated alone."""
+    dims = {"hidden": (0, hidden), "o_in": (1, hidden), "down_in": (2, mlp)}
     out = {}
-    for name, k in (("hidden", hidden), ("o_in", hidden), ("down_in", mlp)):
+    for name in names:
+        idx, k = dims[name]
+        rng = _rng(4, tokens, k, idx)
         m = channel_magnitudes(rng, k, 0.7, outlier_gain=(10.0, 50.0))
         out[name] = random_activations(rng, tokens, m)
     return out

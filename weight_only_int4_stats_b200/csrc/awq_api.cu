@@ -111,9 +111,13 @@ awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_ro
                       awq::kTcBM, 12, false))
       return AWQ_ERR_CUDA;
   }
-  dim3 grid(static_cast<unsigned>((M + BN - 1) / BN),
-            static_cast<unsigned>((a_rows + awq::kTcBM - 1) / awq::kTcBM));
-  kern<<<grid, awq::kTcThreads, L::kSmem, st>>>(tx, ta, args);
+  awq::TcArgs a = args;
+  a.m_tiles = static_cast<int>((M + BN - 1) / BN);
+  a.row_tiles = static_cast<int>((a_rows + awq::kTcBM - 1) / awq::kTcBM);
+  a.rows_total = a_rows;
+  const int64_t blocks = static_cast<int64_t>(a.m_tiles) * a.row_tiles;
+  if (blocks > 0x7FFFFFFFLL) return AWQ_ERR_INVALID_ARG;
+  kern<<<static_cast<unsigned>(blocks), awq::kTcThreads, L::kSmem, st>>>(tx, ta, a);
   return launch_status();
 }
 
@@ -332,16 +336,18 @@ awq_status awq_quantize_pack(const awq_f16* W, int64_t N, int64_t K, const float
 // ------------------------------------------------------------------ search
 namespace {
 struct SearchWs {
-  size_t table, err, part, total;
+  size_t table, inv, err, part, rows, total;
 };
 SearchWs search_ws_layout(int64_t M, int64_t N, int64_t K, int n_alpha) {
   const int64_t N_pad = round_up(N, awq::kTcBM);
   const int64_t m_tiles = (M + tc_bn_for(M) - 1) / tc_bn_for(M);
   SearchWs w;
   w.table = 0;
-  w.err = align256(static_cast<size_t>(n_alpha) * K * sizeof(float));
+  w.inv = align256(static_cast<size_t>(n_alpha) * K * sizeof(float));
+  w.err = w.inv + align256(static_cast<size_t>(n_alpha) * K * sizeof(float));
   w.part = w.err + align256(static_cast<size_t>(n_alpha) * N_pad * K * sizeof(__half));
-  w.total = w.part + align256(static_cast<size_t>(n_alpha) * N_pad * m_tiles * sizeof(double));
+  w.rows = w.part + align256(static_cast<size_t>(n_alpha) * N_pad * m_tiles * sizeof(double));
+  w.total = w.rows + align256(static_cast<size_t>(n_alpha) * N * sizeof(double));
   return w;
 }
 }  // namespace
@@ -388,14 +394,20 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
     if ((s = launch_status()) != AWQ_OK) return s;
     S = table;
   }
+  float* inv = reinterpret_cast<float*>(ws + lay.inv);
+  {
+    const int64_t total = static_cast<int64_t>(n_alpha) * K;
+    awq::inv_table_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(S, total, inv);
+    if ((s = launch_status()) != AWQ_OK) return s;
+  }
   {
     dim3 g(static_cast<unsigned>(N_pad / awq::kQuantRowsPerCta),
            static_cast<unsigned>(K / awq::kGroup), static_cast<unsigned>(n_alpha));
     const __half* w = reinterpret_cast<const __half*>(W);
     if (bits == 4)
-      awq::search_build_error_kernel<4><<<g, 256, 0, st>>>(w, N, K, N_pad, S, E);
+      awq::search_build_error_kernel<4><<<g, 256, 0, st>>>(w, N, K, N_pad, S, inv, E);
     else
-      awq::search_build_error_kernel<3><<<g, 256, 0, st>>>(w, N, K, N_pad, S, E);
+      awq::search_build_error_kernel<3><<<g, 256, 0, st>>>(w, N, K, N_pad, S, inv, E);
     if ((s = launch_status()) != AWQ_OK) return s;
   }
   {
@@ -410,8 +422,15 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
                                                   n_alpha * N_pad, args, st);
     if (s != AWQ_OK) return s;
   }
-  awq::search_reduce_kernel<<<n_alpha, awq::kReduceThreads, 0, st>>>(part, N, N_pad, m_tiles,
-                                                                     row_losses, losses);
+  double* rl = row_losses != nullptr ? row_losses : reinterpret_cast<double*>(ws + lay.rows);
+  {
+    const int64_t n = static_cast<int64_t>(n_alpha) * N;
+    awq::search_row_loss_kernel<<<static_cast<unsigned>((n + awq::kReduceThreads - 1) /
+                                                        awq::kReduceThreads),
+                                  awq::kReduceThreads, 0, st>>>(part, N, N_pad, n_alpha, m_tiles, rl);
+    if ((s = launch_status()) != AWQ_OK) return s;
+  }
+  awq::search_reduce_kernel<<<n_alpha, awq::kReduceThreads, 0, st>>>(rl, N, losses);
   if ((s = launch_status()) != AWQ_OK) return s;
   awq::search_pick_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(
       losses, n_alpha, S, K, best_idx, best_s);

@@ -18,7 +18,8 @@
 //               afterwards the same four warps run the epilogue (tcgen05.ld of their
 //               32-lane quarter of TMEM).
 // Epilogues: fp16 store of Y[m, n], or (search) each weight row's sum over the tile's
-// tokens of the squared output, written as one fp64 partial per (row, token tile).
+// tokens of the squared output, written as one fp64 partial per (token tile, row).
+// Tiles are visited in a grouped order (see tile_of_block) for L2 reuse.
 // Every mbarrier wait is bounded; a timeout sets the device status word and the roles
 // leave their loops so the CTA still releases its TMEM and exits.
 #pragma once
@@ -65,9 +66,27 @@ struct TcArgs {
   const __half* scales; // [K/128, N] (packed source)
   const uint8_t* zeros; // [K/128, N]
   __half* Y;            // [M, N] (store epilogue)
-  double* row_part;     // [rows_total, m_tiles] (search epilogue)
+  double* row_part;     // [m_tiles, rows_total] (search epilogue)
   int m_tiles;
+  int row_tiles;        // 128-row tiles of the A matrix
+  int64_t rows_total;   // rows of the A matrix (row_tiles * 128 for the search)
 };
+
+// Grouped tile order: consecutive CTAs sweep the token tiles of a group of kTcRasterRows
+// weight-row tiles, so the CTAs resident at one time share a few A tiles and a few X tiles
+// in L2 instead of each streaming its own X tile from HBM.
+constexpr int kTcRasterRows = 16;
+
+__device__ __forceinline__ void tile_of_block(int64_t bid, int row_tiles, int m_tiles,
+                                              int& row_tile, int& m_tile) {
+  const int64_t per_group = static_cast<int64_t>(kTcRasterRows) * m_tiles;
+  const int64_t group = bid / per_group;
+  const int64_t in_group = bid % per_group;
+  const int first = static_cast<int>(group) * kTcRasterRows;
+  const int rows_here = row_tiles - first < kTcRasterRows ? row_tiles - first : kTcRasterRows;
+  row_tile = first + static_cast<int>(in_group % rows_here);
+  m_tile = static_cast<int>(in_group / rows_here);
+}
 
 // Dequantize one 4-bit packed word (8 consecutive k) to four fp16 pairs (q - z) * sc.
 __device__ __forceinline__ uint4 dequant_word_scaled(uint32_t w, __half2 bias_lo,
@@ -130,8 +149,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m_tile = blockIdx.x;
-  const int row_tile = blockIdx.y;
+  int m_tile, row_tile;
+  tile_of_block(blockIdx.x, args.row_tiles, args.m_tiles, row_tile, m_tile);
   const int64_t m0 = static_cast<int64_t>(m_tile) * BN;
   const int64_t row0 = static_cast<int64_t>(row_tile) * kTcBM;   // row in the A matrix
   const int nkb = static_cast<int>(args.K / kTcBK);
@@ -306,7 +325,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (kEpi == Epi::kRowSumSq) {
       if (half == 1) red[row] = sumsq;
       named_bar_sync(1, kTcBuilders * 32);
-      if (half == 0 && ok) args.row_part[arow * args.m_tiles + m_tile] = sumsq + red[row];
+      if (half == 0 && ok)
+        args.row_part[static_cast<int64_t>(m_tile) * args.rows_total + arow] = sumsq + red[row];
     }
   }
 

@@ -9,10 +9,10 @@
 //   scale = max((mx - mn) / qmax, 1e-5) rounded to fp16 -> sc;
 //   z = clamp(rint(-mn / sc), 0, qmax);  q = clamp(rint(w' / sc) + z, 0, qmax).
 //
-// One warp owns one (row, group): lane l holds k = 128 j + 4 l .. 4 l + 3, the group's min
-// and max come from five xor-shuffles each, and the packed words are assembled with
-// xor-shuffle ORs between the lanes that share a word. A CTA of 8 warps covers 32 rows of
-// one group so that the [G, N] scales and zeros leave as contiguous runs.
+// Eight lanes own one (row, group): lane l holds 16 consecutive k, the group's min and max
+// come from three xor-shuffles each, and each lane assembles its own packed words (4-bit:
+// two whole words; 3-bit: one low-bit word, and the bit-2 word with one shuffle). A CTA of
+// 8 warps covers 32 rows of one group so the [G, N] scales and zeros leave as contiguous runs.
 #pragma once
 #include "common.cuh"
 
@@ -20,53 +20,87 @@ namespace awq {
 
 constexpr int kQuantRowsPerCta = 32;
 
-struct GroupQuant {
-  float q[4];     // codes of this lane's 4 elements, as exact small integers
+// One (row, group) per 8 lanes: lane sub = lane % 8 holds k = 128 j + 16 sub .. + 15.
+struct QuantGroup {
   float sc;       // fp16-rounded scale, widened
   float z;        // zero point
+  float rcp;      // correctly rounded 1 / sc
   __half sc_h;
 };
 
-template <int kBits>
-__device__ __forceinline__ GroupQuant quantize_lane(const float (&w)[4]) {
-  constexpr float qmax = static_cast<float>((1 << kBits) - 1);
-  float mx = fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3]));
-  float mn = fminf(fminf(w[0], w[1]), fminf(w[2], w[3]));
+__device__ __forceinline__ void load16(const __half* __restrict__ W, int64_t K, int64_t n,
+                                       int64_t k0, bool valid, const float* __restrict__ s,
+                                       float (&w)[16], float (&w_raw)[16]) {
+  uint4 u[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+  if (valid) {
+    const uint4* p = reinterpret_cast<const uint4*>(W + n * K + k0);
+    u[0] = p[0];
+    u[1] = p[1];
+  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t v[4] = {u[h].x, u[h].y, u[h].z, u[h].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(u32_as_h2(v[i]));
+      w_raw[8 * h + 2 * i] = f.x;
+      w_raw[8 * h + 2 * i + 1] = f.y;
+    }
+  }
+  if (s != nullptr) {
+    const float4* sp = reinterpret_cast<const float4*>(s + k0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 sv = sp[q];
+      w[4 * q + 0] = __fmul_rn(w_raw[4 * q + 0], sv.x);
+      w[4 * q + 1] = __fmul_rn(w_raw[4 * q + 1], sv.y);
+      w[4 * q + 2] = __fmul_rn(w_raw[4 * q + 2], sv.z);
+      w[4 * q + 3] = __fmul_rn(w_raw[4 * q + 3], sv.w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = w_raw[i];
+  }
+}
+
+// Group min/max over the 8 lanes of a (row, group) and the group's scale and zero point.
+template <int kBits>
+__device__ __forceinline__ QuantGroup group_params(const float (&w)[16]) {
+  constexpr float qmax = static_cast<float>((1 << kBits) - 1);
+  float mx = w[0], mn = w[0];
+#pragma unroll
+  for (int i = 1; i < 16; ++i) {
+    mx = fmaxf(mx, w[i]);
+    mn = fminf(mn, w[i]);
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
   }
-  GroupQuant g;
+  QuantGroup g;
   float scale = __fdiv_rn(__fsub_rn(mx, mn), qmax);
   scale = fmaxf(scale, 1e-5f);
   g.sc_h = __float2half_rn(scale);
   g.sc = __half2float(g.sc_h);
   g.z = fminf(fmaxf(rintf(__fdiv_rn(-mn, g.sc)), 0.0f), qmax);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    g.q[i] = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w[i], g.sc)), g.z), 0.0f), qmax);
+  g.rcp = __frcp_rn(g.sc);
   return g;
 }
 
-// Loads this lane's 4 weights of (row, group) and applies the per-channel scale.
-__device__ __forceinline__ void load_scaled(const __half* __restrict__ W, int64_t K, int64_t n,
-                                            int64_t k0, const float* __restrict__ s,
-                                            float (&w)[4], float (&w_raw)[4]) {
-  const uint2 raw = *reinterpret_cast<const uint2*>(W + n * K + k0);
-  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-  w_raw[0] = a.x; w_raw[1] = a.y; w_raw[2] = b.x; w_raw[3] = b.y;
-  if (s != nullptr) {
-    const float4 sv = *reinterpret_cast<const float4*>(s + k0);
-    w[0] = __fmul_rn(w_raw[0], sv.x);
-    w[1] = __fmul_rn(w_raw[1], sv.y);
-    w[2] = __fmul_rn(w_raw[2], sv.z);
-    w[3] = __fmul_rn(w_raw[3], sv.w);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) w[i] = w_raw[i];
-  }
+// q = clamp(rint(w' / sc) + z, 0, qmax) with the IEEE quotient. rint of the correctly rounded
+// quotient can only differ from rint of a nearby value where the two straddle a half-integer,
+// so the product w' * rcp (within 2^-22 relative of the exact quotient) decides the code
+// unless it lies within a safe margin of a half-integer; only then is the quotient formed
+// with an IEEE division.
+template <int kBits>
+__device__ __forceinline__ float code_of(float wp, const QuantGroup& g) {
+  constexpr float qmax = static_cast<float>((1 << kBits) - 1);
+  const float t = __fmul_rn(wp, g.rcp);
+  float r = rintf(t);
+  const float gap = fabsf(fabsf(__fsub_rn(t, r)) - 0.5f);
+  if (gap <= fmaxf(fabsf(t), 1.0f) * 0x1p-18f) r = rintf(__fdiv_rn(wp, g.sc));
+  return fminf(fmaxf(__fadd_rn(r, g.z), 0.0f), qmax);
 }
 
 // 4-bit: k-offset o of a word sits in nibble position o/2 + 4*(o%2).
@@ -80,52 +114,47 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
   __shared__ uint8_t sh_zero[kQuantRowsPerCta];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const int sub = lane & 7;
+  const int lr = 4 * warp + (lane >> 3);                 // local row 0..31
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * kQuantRowsPerCta + lr;
+  const bool valid = n < N;
   const int64_t j = blockIdx.y;                          // group index
-  const int64_t k0 = j * kGroup + 4 * lane;
-  const int64_t words_per_row = (kBits == 4) ? K / 8 : 3 * K / 32;
-#pragma unroll 1
-  for (int rr = 0; rr < kQuantRowsPerCta / 8; ++rr) {
-    const int lr = warp * (kQuantRowsPerCta / 8) + rr;  // local row 0..31
-    const int64_t n = static_cast<int64_t>(blockIdx.x) * kQuantRowsPerCta + lr;
-    if (n >= N) break;                                   // warp-uniform
-    float w[4], w_raw[4];
-    load_scaled(W, K, n, k0, s, w, w_raw);
-    const GroupQuant g = quantize_lane<kBits>(w);
-    if (kBits == 4) {
-      uint32_t part = 0;
+  const int64_t k0 = j * kGroup + 16 * sub;
+  float w[16], w_raw[16];
+  load16(W, K, n, k0, valid, s, w, w_raw);
+  const QuantGroup g = group_params<kBits>(w);
+  uint32_t q[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int o = 4 * (lane & 1) + i;
-        part |= static_cast<uint32_t>(g.q[i]) << (4 * nibble_pos(o));
-      }
-      part |= __shfl_xor_sync(0xffffffffu, part, 1);
-      if ((lane & 1) == 0) qweight[n * words_per_row + j * 16 + (lane >> 1)] = part;
-    } else {
-      uint32_t p0 = 0, p1 = 0, p2 = 0;
+  for (int i = 0; i < 16; ++i) q[i] = static_cast<uint32_t>(code_of<kBits>(w[i], g));
+  if (kBits == 4) {
+    uint32_t w0 = 0, w1 = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int o = 4 * (lane & 7) + i;                // offset inside the 32-k block
-        const uint32_t q = static_cast<uint32_t>(g.q[i]);
-        const int oo = o & 15;
-        const uint32_t lo = (q & 3u) << (2 * ((oo >> 1) + 8 * (oo & 1)));
-        if (o < 16) p0 |= lo; else p1 |= lo;
-        p2 |= ((q >> 2) & 1u) << ((o >> 1) + 16 * (o & 1));
-      }
-#pragma unroll
-      for (int m = 1; m < 8; m <<= 1) {
-        p0 |= __shfl_xor_sync(0xffffffffu, p0, m);
-        p1 |= __shfl_xor_sync(0xffffffffu, p1, m);
-        p2 |= __shfl_xor_sync(0xffffffffu, p2, m);
-      }
-      if ((lane & 7) == 0) {
-        uint32_t* dst = qweight + n * words_per_row + (j * 4 + (lane >> 3)) * 3;
-        dst[0] = p0; dst[1] = p1; dst[2] = p2;
-      }
+    for (int o = 0; o < 8; ++o) {
+      w0 |= q[o] << (4 * nibble_pos(o));
+      w1 |= q[8 + o] << (4 * nibble_pos(o));
     }
-    if (lane == 0) {
-      sh_scale[lr] = g.sc_h;
-      sh_zero[lr] = static_cast<uint8_t>(g.z);
+    if (valid)
+      *reinterpret_cast<uint2*>(qweight + n * (K / 8) + j * 16 + 2 * sub) = make_uint2(w0, w1);
+  } else {
+    // lanes sub = 2b + h hold offsets 16h..16h+15 of the group's 32-k block b
+    const int h = sub & 1;
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int o = 16 * h + e;                          // offset inside the 32-k block
+      lo |= (q[e] & 3u) << (2 * ((e >> 1) + 8 * (e & 1)));
+      hi |= ((q[e] >> 2) & 1u) << ((o >> 1) + 16 * (o & 1));
     }
+    hi |= __shfl_xor_sync(0xffffffffu, hi, 1);
+    if (valid) {
+      uint32_t* dst = qweight + n * (3 * K / 32) + (j * 4 + (sub >> 1)) * 3;
+      dst[h] = lo;
+      if (h == 0) dst[2] = hi;
+    }
+  }
+  if (sub == 0) {
+    sh_scale[lr] = g.sc_h;
+    sh_zero[lr] = static_cast<uint8_t>(g.z);
   }
   __syncthreads();
   const int t = threadIdx.x;
@@ -135,44 +164,63 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
     zeros[j * N + nb + t - 32] = sh_zero[t - 32];
 }
 
-// Search operand: for grid point a, E[a][n][k] = fp16(deq[n,k] * (1 / s_a[k]) - w[n,k]) with
-// deq = (q - z) * sc from the quantizer above; rows N..N_pad-1 are written as zeros so that
-// 128-row tiles never straddle two grid points.
+// Search operand: for grid point a, E[a][n][k] = fp16(deq[n,k] * inv_a[k] - w[n,k]) with
+// deq = (q - z) * sc from the quantizer above and inv_a = 1 / s_a (correctly rounded, from
+// a table); rows N..N_pad-1 are written as zeros so that 128-row tiles never straddle two
+// grid points.
 template <int kBits>
 __global__ void __launch_bounds__(256) search_build_error_kernel(
     const __half* __restrict__ W, int64_t N, int64_t K, int64_t N_pad,
-    const float* __restrict__ s_table, __half* __restrict__ E) {
+    const float* __restrict__ s_table, const float* __restrict__ inv_table,
+    __half* __restrict__ E) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const int sub = lane & 7;
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * kQuantRowsPerCta + 4 * warp + (lane >> 3);
   const int64_t j = blockIdx.y;
   const int64_t a = blockIdx.z;
-  const int64_t k0 = j * kGroup + 4 * lane;
+  const int64_t k0 = j * kGroup + 16 * sub;
   const float* s = s_table + a * K;
-  __half* Ea = E + a * N_pad * K;
-#pragma unroll 1
-  for (int rr = 0; rr < kQuantRowsPerCta / 8; ++rr) {
-    const int64_t n = static_cast<int64_t>(blockIdx.x) * kQuantRowsPerCta +
-                      warp * (kQuantRowsPerCta / 8) + rr;
-    if (n >= N_pad) break;
-    uint2 out = make_uint2(0u, 0u);
-    if (n < N) {
-      float w[4], w_raw[4];
-      load_scaled(W, K, n, k0, s, w, w_raw);
-      const GroupQuant g = quantize_lane<kBits>(w);
-      const float4 sv = *reinterpret_cast<const float4*>(s + k0);
-      const float sa[4] = {sv.x, sv.y, sv.z, sv.w};
-      __half e[4];
+  const bool valid = n < N;
+  float w[16], w_raw[16];
+  load16(W, K, n, k0, valid, s, w, w_raw);
+  const QuantGroup g = group_params<kBits>(w);
+  if (n >= N_pad) return;
+  uint4 out[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+  if (valid) {
+    const float4* ip = reinterpret_cast<const float4*>(inv_table + a * K + k0);
+    float inv[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float deq = __fmul_rn(__fsub_rn(g.q[i], g.z), g.sc);
-        const float inv = __fdiv_rn(1.0f, sa[i]);
-        e[i] = __float2half_rn(__fsub_rn(__fmul_rn(deq, inv), w_raw[i]));
-      }
-      out.x = h2_as_u32(__halves2half2(e[0], e[1]));
-      out.y = h2_as_u32(__halves2half2(e[2], e[3]));
+    for (int qd = 0; qd < 4; ++qd) {
+      const float4 v = ip[qd];
+      inv[4 * qd] = v.x; inv[4 * qd + 1] = v.y; inv[4 * qd + 2] = v.z; inv[4 * qd + 3] = v.w;
     }
-    *reinterpret_cast<uint2*>(Ea + n * K + k0) = out;
+    uint32_t e2[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float e[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int idx = 2 * i + u;
+        const float q = code_of<kBits>(w[idx], g);
+        const float deq = __fmul_rn(__fsub_rn(q, g.z), g.sc);
+        e[u] = __fsub_rn(__fmul_rn(deq, inv[idx]), w_raw[idx]);
+      }
+      e2[i] = h2_as_u32(__floats2half2_rn(e[0], e[1]));
+    }
+    out[0] = make_uint4(e2[0], e2[1], e2[2], e2[3]);
+    out[1] = make_uint4(e2[4], e2[5], e2[6], e2[7]);
   }
+  uint4* dst = reinterpret_cast<uint4*>(E + a * N_pad * K + n * K + k0);
+  dst[0] = out[0];
+  dst[1] = out[1];
+}
+
+// inv_table[a][k] = 1 / s_table[a][k], correctly rounded.
+__global__ void inv_table_kernel(const float* __restrict__ s_table, int64_t total,
+                                 float* __restrict__ inv_table) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < total) inv_table[i] = __frcp_rn(s_table[i]);
 }
 
 // s_table[a][k] = (float) pow((double) max(s_x[k], 1e-4f), (double) alphas[a]).

@@ -10,21 +10,29 @@ namespace awq {
 
 constexpr int kReduceThreads = 256;
 
-// One CTA per grid point a: row_loss[n] = sum over token tiles (in order); thread t adds
-// rows t, t+256, ... in order; the 256 thread sums are combined by a fixed binary tree.
+// Per-row losses: row r of grid point a adds its token-tile partials in tile order
+// (partials are stored token-tile-major, so consecutive threads read consecutive rows).
+__global__ void __launch_bounds__(kReduceThreads) search_row_loss_kernel(
+    const double* __restrict__ row_part, int64_t N, int64_t N_pad, int n_alpha, int m_tiles,
+    double* __restrict__ row_loss /*[n_alpha, N]*/) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<int64_t>(n_alpha) * N) return;
+  const int64_t a = i / N, n = i % N;
+  const int64_t rows_total = static_cast<int64_t>(n_alpha) * N_pad;
+  const double* p = row_part + a * N_pad + n;
+  double r = 0.0;
+  for (int j = 0; j < m_tiles; ++j) r += p[static_cast<int64_t>(j) * rows_total];
+  row_loss[i] = r;
+}
+
+// One CTA per grid point a: the N row losses are added by thread t in the order
+// t, t+256, ... and the 256 thread sums by a fixed binary tree.
 __global__ void __launch_bounds__(kReduceThreads) search_reduce_kernel(
-    const double* __restrict__ row_part, int64_t N, int64_t N_pad, int m_tiles,
-    double* __restrict__ row_losses, double* __restrict__ losses) {
+    const double* __restrict__ row_loss, int64_t N, double* __restrict__ losses) {
   const int a = blockIdx.x;
   const int t = threadIdx.x;
   double acc = 0.0;
-  for (int64_t n = t; n < N; n += kReduceThreads) {
-    const double* p = row_part + (static_cast<int64_t>(a) * N_pad + n) * m_tiles;
-    double r = 0.0;
-    for (int j = 0; j < m_tiles; ++j) r += p[j];
-    if (row_losses != nullptr) row_losses[static_cast<int64_t>(a) * N + n] = r;
-    acc += r;
-  }
+  for (int64_t n = t; n < N; n += kReduceThreads) acc += row_loss[static_cast<int64_t>(a) * N + n];
   __shared__ double red[kReduceThreads];
   red[t] = acc;
   __syncthreads();
