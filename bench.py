@@ -287,44 +287,61 @@ def decoder_layer_rows(awq, dev, pk):
     torch.cuda.empty_cache()
 
     # the whole layer as one pipeline: stats -> 4 searches -> 7 packs -> 7 GEMMs over the batch
+    # (outputs and workspaces allocated before the timed region)
+    Mtok = int(Xd["hidden"].shape[0])
+    y_buf = torch.empty(Mtok * max(W.shape[0] for W in Wd.values()), dtype=torch.float16,
+                        device=dev)
+    g_ws = torch.empty(awq.lib().awq_gemm_workspace_size(Mtok, 1, max(W.shape[1] for W in
+                                                                       Wd.values()), 4),
+                       dtype=torch.uint8, device=dev)
     jobs = [("hidden", ["q_proj", "k_proj", "v_proj"]), ("hidden", ["gate_proj", "up_proj"]),
             ("o_in", ["o_proj"]), ("down_in", ["down_proj"])]
-    torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    chosen = {}
+    search_flops = 0
+    stacked = {tuple(names): (torch.cat([Wd[n] for n in names]).contiguous() if len(names) > 1
+                              else Wd[names[0]]) for _, names in jobs}
+    ws_bytes = max(awq.lib().awq_search_scale_workspace_size(Xd[x].shape[0], W.shape[0],
+                                                            W.shape[1], 20)
+                   for (x, names), W in zip(jobs, stacked.values()))
+    search_ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
     ev[0].record()
     stats = {name: awq.awq_act_stats(Xd[name]) for name in ("hidden", "o_in", "down_in")}
     ev[1].record()
-    chosen = {}
-    search_flops = 0
     for xname, names in jobs:
-        W = torch.cat([Wd[n] for n in names]).contiguous() if len(names) > 1 else Wd[names[0]]
-        _, best, best_s, _ = awq.awq_search_scale(W, Xd[xname], stats[xname], alphas, 4)
+        W = stacked[tuple(names)]
+        _, best, best_s, _ = awq.awq_search_scale(W, Xd[xname], stats[xname], alphas, 4,
+                                                  workspace=search_ws)
         search_flops += 20 * 2 * Xd[xname].shape[0] * W.shape[0] * W.shape[1]
         for n in names:
             chosen[n] = (best, best_s)
-        del W
     ev[2].record()
     packed = {n: awq.awq_quantize_pack(Wd[n], chosen[n][1], 4) for n in Wd}
     ev[3].record()
     gemm_flops = 0
     xin = {"q_proj": "hidden", "k_proj": "hidden", "v_proj": "hidden", "gate_proj": "hidden",
            "up_proj": "hidden", "o_proj": "o_in", "down_proj": "down_in"}
+    invs = {n: (1.0 / chosen[n][1]).contiguous() for n in packed}
+    ev3b = torch.cuda.Event(enable_timing=True)
+    ev3b.record()
     for n, (qw, sc, z) in packed.items():
         N, K = Wd[n].shape
-        inv = (1.0 / chosen[n][1]).contiguous()
-        Y = awq.awq_gemm_w4a16(Xd[xin[n]], qw, sc, z, N, K, 4, inv_s=inv)
-        gemm_flops += 2 * Xd[xin[n]].shape[0] * N * K
-        del Y
+        Y = y_buf[:Mtok * N].view(Mtok, N)
+        awq.awq_gemm_w4a16(Xd[xin[n]], qw, sc, z, N, K, 4, inv_s=invs[n], out=Y, workspace=g_ws)
+        gemm_flops += 2 * Mtok * N * K
     ev[4].record()
     torch.cuda.synchronize()
     st = [ev[i].elapsed_time(ev[i + 1]) / 1e3 for i in range(4)]
+    st_gemm_only = ev3b.elapsed_time(ev[4]) / 1e3
     rows["decoder_layer_pipeline"] = {
         "tokens": int(Xd["hidden"].shape[0]), "seconds": sum(st),
         "act_stats_s": st[0], "search_s": st[1], "pack_s": st[2], "gemm_s": st[3],
-        "search_TFLOP/s": search_flops / st[1] / 1e12, "gemm_TFLOP/s": gemm_flops / st[3] / 1e12,
+        "search_TFLOP/s": search_flops / st[1] / 1e12,
+        "gemm_TFLOP/s": gemm_flops / st_gemm_only / 1e12,
         "alpha_index": {n: int(chosen[n][0].item()) for n in chosen},
     }
-    del Xd, Wd, packed, stats, chosen
+    del Xd, Wd, packed, stats, chosen, stacked, search_ws, y_buf, g_ws
     torch.cuda.empty_cache()
 
     # quantize-and-pack on the largest prefill weight (HBM-bound)
@@ -485,6 +502,32 @@ def run_b200(args, world, rank, local):
     del shapes
     torch.cuda.empty_cache()
 
+    # ---- batched decode / small prefill: M in 32..256 on the batched shapes (weights > L2 in
+    #      rotation), GB/s and TFLOP/s per (shape, M)
+    batched = []
+    for (N, K) in (synth.BATCHED_SHAPES if args.only == "all" else []):
+        W, mag, X = synth.batched_layer(N, K)
+        s_ = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(dev)
+        Wt = torch.from_numpy(W).to(dev)
+        base = awq.awq_quantize_pack(Wt, s_, 4)
+        del Wt
+        per = sum(t.numel() * t.element_size() for t in base)
+        ncp = max(2, math.ceil(2 * l2 / per))
+        cps = [base] + [tuple(t.clone() for t in base) for _ in range(ncp - 1)]
+        Xt = torch.from_numpy(X).to(dev)
+        Yt = torch.empty(X.shape[0], N, dtype=torch.float16, device=dev)
+        for M in synth.BATCHED_M:
+            f = (lambda r, M=M: awq.awq_gemm_w4a16(Xt[:M], *cps[r % ncp], N, K, 4, out=Yt[:M]))
+            f(0)
+            t = time_steps(f, 100, 5, stream, world)
+            b = gemm_bytes(M, N, K)
+            batched.append({"N": N, "K": K, "M": M, "us": t / 100 * 1e6,
+                            "GB/s": b * 100 / t / 1e9, "TFLOP/s": 2 * M * N * K * 100 / t / 1e12,
+                            "frac_hbm": b * 100 / t / 1e9 / pk["hbm_gbs"],
+                            "frac_tensor": 2 * M * N * K * 100 / t / 1e12 / pk["bf16_tflops"]})
+        del cps, base, Xt, Yt
+        torch.cuda.empty_cache()
+
     # ---- prefill at M = 2048 (4-bit on the three shapes, then the 3-bit variant)
     prefill = []
     pf_cases = [(N, K, 4) for (N, K) in synth.PREFILL_SHAPES] + [(*synth.PREFILL_SHAPES[0], 3)]
@@ -542,6 +585,7 @@ def run_b200(args, world, rank, local):
                     "frac": pf_value / pk["bf16_tflops"] if prefill else None,
                     "kernel": "tc_gemm_kernel"},
         "sweep": sweep,
+        "batched": batched,
         "rows": rows,
         "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": cpu_desc, "seconds": cpu_t},

@@ -77,6 +77,13 @@ AWQ_API int awq_abi_version(void);
  * last check, AWQ_ERR_CUDA if the synchronisation failed, AWQ_OK otherwise. */
 AWQ_API awq_status awq_check_error(void* stream);
 
+/* Self-test of failure detection: launches one thread that waits on a barrier nothing ever
+ * arrives on, with a 50 ms limit instead of the usual ~2 s, so the wait runs out the way a
+ * stalled pipeline stage would. The kernel writes 1 to *waited_out (a device int) when its
+ * wait ran out, sets the device status word, and returns; the next awq_check_error() on
+ * the stream returns AWQ_ERR_TIMEOUT and the context stays usable. */
+AWQ_API awq_status awq_selftest_timeout(int* waited_out, void* stream);
+
 /* ---------------------------------------------------------------- activation statistics
  * robotsatlas.com "AWQ", "How it works" / "Components: Activation saliency analysis":
  * the activation magnitude of every input channel on the calibration set,

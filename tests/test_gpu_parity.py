@@ -170,6 +170,16 @@ def test_gemm_tensor_core(awq, M, N, K, bits):
     _check_gemm(awq, X, qw, sc, z, N, K, bits)
 
 
+@pytest.mark.parametrize("bits", [4, 3])
+@pytest.mark.parametrize("M,N,K", [(17, 130, 1024), (33, 258, 2048), (100, 1000, 4096)])
+def test_gemm_split_k_ragged(awq, M, N, K, bits):
+    # few output tiles -> the K range is split across CTAs and the fp32 partial sums are
+    # reduced afterwards (including an M*N that is not a multiple of 4)
+    W, X, m = rand_layer(M + N + K + bits, N, K, M)
+    qw, sc, z = _packed(W, np.sqrt(m).astype(np.float32), bits)
+    _check_gemm(awq, X, qw, sc, z, N, K, bits)
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_gemm_3bit_decode_sizes(awq, M):
     N, K = 320, 768
@@ -338,3 +348,22 @@ def test_decode_chain_output_feeds_next_input(awq):
     o1 = O.gemm_w4a16(X, *p1, N1, K1, 4, 128).astype(np.float16)
     o2 = O.gemm_w4a16(o1, *p2, N2, N1, 4, 128)
     assert rel_fro(Y2.float().cpu().numpy(), o2) <= GEMM_RTOL
+
+
+# ----------------------------------------------------------------------------- failure detection
+
+def test_bounded_wait_times_out_and_reports(awq):
+    # A barrier that nothing arrives on: the kernel's bounded wait must run out, report
+    # AWQ_ERR_TIMEOUT through awq_check_error, and leave the context usable.
+    import ctypes
+    L = awq.lib()
+    flag = torch.zeros(4, dtype=torch.int32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert L.awq_check_error(stream) == 0
+    assert L.awq_selftest_timeout(ctypes.c_void_p(flag.data_ptr()), stream) == 0
+    assert L.awq_check_error(stream) == 5          # AWQ_ERR_TIMEOUT
+    assert int(flag[0].item()) == 1
+    assert L.awq_check_error(stream) == 0          # the status word was cleared
+    W, X, _ = rand_layer(9, 64, 256, 4)            # and the library still computes correctly
+    s = awq.awq_act_stats(cu(X)).cpu().numpy()
+    np.testing.assert_array_equal(s, O.act_stats(X))

@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
             "awq_status_string": (ctypes.c_char_p, [I32]),
             "awq_abi_version": (I32, []),
             "awq_check_error": (I32, [P]),
+            "awq_selftest_timeout": (I32, [P, P]),
             "awq_act_stats_workspace_size": (SZ, [I64, I64]),
             "awq_act_stats": (I32, [P, I64, I64, P, P, SZ, P]),
             "awq_act_stats_noalloc": (I32, [P, I64, I64, P, P]),
@@ -189,8 +190,9 @@ def awq_gemm_w4a16(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
     M = X.shape[0]
     Y = torch.empty(M, N, dtype=torch.float16, device=X.device) if out is None else out
     ws = workspace
-    if ws is None and inv_s is not None:
-        ws = _workspace(lib().awq_gemm_workspace_size(M, N, K, bits), X.device)
+    if ws is None:
+        need = lib().awq_gemm_workspace_size(M, N, K, bits)
+        ws = _workspace(need, X.device) if need > 0 else None
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("awq_gemm_w4a16", lib().awq_gemm_w4a16(
         _ptr(X), M, _ptr(qweight), _ptr(scales), _ptr(zeros), N, K, bits, group, _ptr(inv_s),

@@ -115,7 +115,8 @@ awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_ro
   a.m_tiles = static_cast<int>((M + BN - 1) / BN);
   a.row_tiles = static_cast<int>((a_rows + awq::kTcBM - 1) / awq::kTcBM);
   a.rows_total = a_rows;
-  const int64_t blocks = static_cast<int64_t>(a.m_tiles) * a.row_tiles;
+  if (a.k_splits < 1) a.k_splits = 1;
+  const int64_t blocks = static_cast<int64_t>(a.m_tiles) * a.row_tiles * a.k_splits;
   if (blocks > 0x7FFFFFFFLL) return AWQ_ERR_INVALID_ARG;
   kern<<<static_cast<unsigned>(blocks), awq::kTcThreads, L::kSmem, st>>>(tx, ta, a);
   return launch_status();
@@ -188,6 +189,27 @@ awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweigh
 
 int tc_bn_for(int64_t M) { return M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
+// Split-K for the tensor-core GEMM when the output has too few 128 x BN tiles to occupy the
+// GPU (batched decode, small prefill): fill one wave of resident CTAs, keep at least two
+// groups per slice, and keep the fp32 partial traffic (8 bytes per output and slice) within
+// about the packed weight bytes.
+int splitk_for(int64_t M, int64_t N, int64_t K) {
+  const int64_t bn = tc_bn_for(M);
+  const int64_t tiles = ((N + awq::kTcBM - 1) / awq::kTcBM) * ((M + bn - 1) / bn);
+  const int64_t sms = num_sms();
+  // CTAs of the wider tiles need more than half an SM's shared memory (one per SM); the
+  // split never adds a second wave of CTAs
+  const int64_t resident = sms * (bn <= 32 ? 2 : 1);
+  if (tiles >= sms) return 1;
+  int64_t s = resident / tiles;
+  const int64_t by_groups = (K / awq::kGroup) / 2;
+  const int64_t by_traffic = K / (8 * M);
+  if (s > by_groups) s = by_groups;
+  if (s > by_traffic) s = by_traffic;
+  if (s > 16) s = 16;
+  return s < 2 ? 1 : static_cast<int>(s);
+}
+
 bool bad_dim(int64_t v) { return v < 0 || v > kMaxDim; }
 
 }  // namespace
@@ -218,6 +240,14 @@ awq_status awq_check_error(void* stream) {
     return AWQ_ERR_CUDA;
   if (word & awq::kDevErrTimeout) return AWQ_ERR_TIMEOUT;
   return AWQ_OK;
+}
+
+awq_status awq_selftest_timeout(int* waited_out, void* stream) {
+  if (waited_out == nullptr || (reinterpret_cast<uintptr_t>(waited_out) & 3u) != 0)
+    return AWQ_ERR_INVALID_ARG;
+  awq::timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      50ull * 1000 * 1000, waited_out);
+  return launch_status();
 }
 
 // ------------------------------------------------------------------ act_stats
@@ -418,6 +448,7 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
     args.K = K;
     args.row_part = part;
     args.m_tiles = m_tiles;
+    args.k_splits = 1;
     s = launch_tc_bn<ASrc::kFp16, Epi::kRowSumSq>(reinterpret_cast<const __half*>(X), M, E,
                                                   n_alpha * N_pad, args, st);
     if (s != AWQ_OK) return s;
@@ -439,10 +470,12 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
 
 // ------------------------------------------------------------------ GEMM
 size_t awq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits) {
-  (void)N;
-  if (M <= 0 || K <= 0) return 0;
+  if (M <= 0 || K <= 0 || N <= 0) return 0;
   if (M <= 16 && bits == 4) return 0;
-  return align256(static_cast<size_t>(M) * K * sizeof(__half));
+  const int splits = splitk_for(M, N, K);
+  size_t bytes = align256(static_cast<size_t>(M) * K * sizeof(__half));   // x * inv_s
+  if (splits > 1) bytes += align256(static_cast<size_t>(splits) * M * N * sizeof(float));
+  return bytes;
 }
 
 awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
@@ -479,9 +512,17 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
   }
   if ((N + awq::kTcBM - 1) / awq::kTcBM > 65535) return AWQ_ERR_INVALID_ARG;
   const __half* xop = x;
+  const int splits = splitk_for(M, N, K);
+  const size_t xs_bytes = align256(static_cast<size_t>(M) * K * sizeof(__half));
+  const size_t part_bytes =
+      splits > 1 ? align256(static_cast<size_t>(splits) * M * N * sizeof(float)) : 0;
+  const size_t need = (inv_s != nullptr ? xs_bytes : 0) + part_bytes;
+  if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
+    return AWQ_ERR_WORKSPACE;
+  float* partial = splits > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                        (inv_s != nullptr ? xs_bytes : 0))
+                              : nullptr;
   if (inv_s != nullptr) {
-    const size_t need = align256(static_cast<size_t>(M) * K * sizeof(__half));
-    if (!workspace || ws_bytes < need || !aligned16(workspace)) return AWQ_ERR_WORKSPACE;
     __half* xs = static_cast<__half*>(workspace);
     const int64_t n8 = M * K / 8;
     awq::prescale_x_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, st>>>(x, inv_s, M,
@@ -499,8 +540,16 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
   args.zeros = zeros;
   args.Y = y;
   args.m_tiles = static_cast<int>((M + tc_bn_for(M) - 1) / tc_bn_for(M));
-  if (bits == 3) return launch_tc_bn<ASrc::kPacked3, Epi::kStoreY>(xop, M, qweight, N, args, st);
-  return launch_tc_bn<ASrc::kPacked4, Epi::kStoreY>(xop, M, qweight, N, args, st);
+  args.k_splits = splits;
+  args.partial = partial;
+  awq_status r =
+      bits == 3 ? launch_tc_bn<ASrc::kPacked3, Epi::kStoreY>(xop, M, qweight, N, args, st)
+                : launch_tc_bn<ASrc::kPacked4, Epi::kStoreY>(xop, M, qweight, N, args, st);
+  if (r != AWQ_OK || splits == 1) return r;
+  const int64_t MN = M * N;
+  awq::splitk_reduce_kernel<<<static_cast<unsigned>((MN / 4 + 1 + 255) / 256), 256, 0, st>>>(
+      partial, splits, MN, y);
+  return launch_status();
 }
 
 }  // extern "C"

@@ -69,18 +69,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 
 // Waits for the phase with the given parity to complete. Returns false (and flags the
-// status word) if it did not within kWaitLimitNs; the caller then abandons its work.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// status word) if it did not within `limit_ns` (default kWaitLimitNs); the caller then
+// abandons its work.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(a, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       flag_error(kDevErrTimeout);
       return false;
     }
+  }
+}
+
+// Self-test of the timeout path: one thread waits on an mbarrier that nothing ever arrives
+// on, with a short limit, so the wait runs out, flags the status word and the kernel returns.
+__global__ void timeout_selftest_kernel(unsigned long long limit_ns, int* waited_out) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    const bool ok = mbar_wait(&bar, 0, limit_ns);
+    *waited_out = ok ? 0 : 1;
   }
 }
 

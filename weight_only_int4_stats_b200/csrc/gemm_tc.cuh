@@ -70,6 +70,8 @@ struct TcArgs {
   int m_tiles;
   int row_tiles;        // 128-row tiles of the A matrix
   int64_t rows_total;   // rows of the A matrix (row_tiles * 128 for the search)
+  int k_splits;         // > 1: each CTA covers a group-aligned slice of K (split-K)
+  float* partial;       // [k_splits, M, N] fp32 partial sums (split-K store epilogue)
 };
 
 // Grouped tile order: consecutive CTAs sweep the token tiles of a group of kTcRasterRows
@@ -150,10 +152,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   int m_tile, row_tile;
-  tile_of_block(blockIdx.x, args.row_tiles, args.m_tiles, row_tile, m_tile);
+  const int64_t tiles = static_cast<int64_t>(args.row_tiles) * args.m_tiles;
+  const int ksplit = static_cast<int>(blockIdx.x / tiles);
+  tile_of_block(blockIdx.x % tiles, args.row_tiles, args.m_tiles, row_tile, m_tile);
   const int64_t m0 = static_cast<int64_t>(m_tile) * BN;
   const int64_t row0 = static_cast<int64_t>(row_tile) * kTcBM;   // row in the A matrix
-  const int nkb = static_cast<int>(args.K / kTcBK);
+  // this CTA's K slice, in whole groups of 128 (two 64-wide stages per group)
+  const int G = static_cast<int>(args.K / kGroup);
+  const int kb0 = 2 * static_cast<int>(static_cast<int64_t>(ksplit) * G / args.k_splits);
+  const int kb1 = 2 * static_cast<int>(static_cast<int64_t>(ksplit + 1) * G / args.k_splits);
+  const int nkb = kb1 - kb0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
@@ -182,14 +190,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % kTcStages;
-        const uint32_t ph = (kb / kTcStages) & 1;
-        if (kA == ASrc::kPacked3 && (kb & 1) == 0) {
-          const int pk = kb >> 1, ps = pk % kTcPk3Slots;
-          if (!mbar_wait(&pempty[ps], ((pk / kTcPk3Slots) & 1) ^ 1)) break;
+      for (int i = 0; i < nkb; ++i) {
+        const int kb = kb0 + i;
+        const int s = i % kTcStages;
+        const uint32_t ph = (i / kTcStages) & 1;
+        if (kA == ASrc::kPacked3 && (i & 1) == 0) {
+          const int li = i >> 1, ps = li % kTcPk3Slots;
+          if (!mbar_wait(&pempty[ps], ((li / kTcPk3Slots) & 1) ^ 1)) break;
           mbar_arrive_expect_tx(&pfull[ps], L::kPBytes);
-          tma_load_2d(smem + L::kPOff + ps * L::kPBytes, &tmap_a, &pfull[ps], pk * 12,
+          tma_load_2d(smem + L::kPOff + ps * L::kPBytes, &tmap_a, &pfull[ps], (kb >> 1) * 12,
                       static_cast<int32_t>(row0));
         }
         if (!mbar_wait(&empty[s], ph ^ 1)) break;
@@ -209,9 +218,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = f16_idesc(kTcBM, BN);
       bool ok = true;
-      for (int kb = 0; kb < nkb && ok; ++kb) {
-        const int s = kb % kTcStages;
-        const uint32_t ph = (kb / kTcStages) & 1;
+      for (int i = 0; i < nkb && ok; ++i) {
+        const int s = i % kTcStages;
+        const uint32_t ph = (i / kTcStages) & 1;
         ok = mbar_wait(&full[s], ph);
         if (ok && kPacked) ok = mbar_wait(&built[s], ph);
         if (!ok) break;
@@ -221,7 +230,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kTcBK / 16; ++kk) {
           tc_mma_f16(tmem_d, sw128_kmajor_desc(a_base + kk * 32),
-                     sw128_kmajor_desc(x_base + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+                     sw128_kmajor_desc(x_base + kk * 32), idesc, (i | kk) != 0 ? 1u : 0u);
         }
         tc_commit(&empty[s]);
       }
@@ -236,10 +245,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     if (kPacked) {
       __half2 lo, hi, sc;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % kTcStages;
-        const uint32_t ph = (kb / kTcStages) & 1;
-        if ((kb & 1) == 0) {   // new group of 128: this row's zero point and scale
+      for (int i = 0; i < nkb; ++i) {
+        const int kb = kb0 + i;
+        const int s = i % kTcStages;
+        const uint32_t ph = (i / kTcStages) & 1;
+        if ((i & 1) == 0) {    // new group of 128: this row's zero point and scale
           const int64_t g = kb >> 1;
           const uint32_t z = n < N ? args.zeros[g * N + n] : 0u;
           const __half sv = n < N ? args.scales[g * N + n] : __float2half(0.0f);
@@ -248,8 +258,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           sc = __half2half2(sv);
         }
         bool got = mbar_wait(&full[s], ph) && mbar_wait(&empty[s], ph ^ 1);
-        const int pk = kb >> 1, ps = pk % kTcPk3Slots;
-        if (kA == ASrc::kPacked3 && got) got = mbar_wait(&pfull[ps], (pk / kTcPk3Slots) & 1);
+        const int li = i >> 1, ps = li % kTcPk3Slots;
+        if (kA == ASrc::kPacked3 && got) got = mbar_wait(&pfull[ps], (li / kTcPk3Slots) & 1);
         ok = __all_sync(0xffffffffu, got);   // keep the warp converged for .aligned ops
         if (!ok) break;
         uint8_t* atile = smem + L::kAOff + s * L::kABytes;
@@ -264,7 +274,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         } else {
           const uint32_t* pw = reinterpret_cast<const uint32_t*>(
-              smem + L::kPOff + ps * L::kPBytes + r * 48 + 12 * (2 * (kb & 1) + h));
+              smem + L::kPOff + ps * L::kPBytes + r * 48 + 12 * (2 * (i & 1) + h));
           const uint32_t w0 = pw[0], w1 = pw[1], w2s = pw[2];
           uint4 o;
 #define AWQ_DQ3_CHUNK(I)                                                   \
@@ -278,7 +288,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           AWQ_DQ3_CHUNK(2)
           AWQ_DQ3_CHUNK(3)
 #undef AWQ_DQ3_CHUNK
-          if (kb & 1) mbar_arrive(&pempty[ps]);   // both stages of the group are built
+          if (i & 1) mbar_arrive(&pempty[ps]);    // both stages of the group are built
         }
         fence_proxy_async_smem();
         mbar_arrive(&built[s]);
@@ -305,10 +315,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_ld_wait();
         if (kEpi == Epi::kStoreY) {
           if (arow < args.N) {
+            if (args.k_splits == 1) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int64_t m = m0 + col + j;
-              if (m < args.M) args.Y[m * args.N + arow] = __float2half_rn(__uint_as_float(v[j]));
+              for (int j = 0; j < 16; ++j) {
+                const int64_t m = m0 + col + j;
+                if (m < args.M) args.Y[m * args.N + arow] = __float2half_rn(__uint_as_float(v[j]));
+              }
+            } else {
+              float* P = args.partial + static_cast<int64_t>(ksplit) * args.M * args.N;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int64_t m = m0 + col + j;
+                if (m < args.M) P[m * args.N + arow] = __uint_as_float(v[j]);
+              }
             }
           }
         } else {
@@ -335,6 +354,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_d, L::kTmemCols);
+  }
+}
+
+// Y[m, n] = fp16(sum over the K slices of the fp32 partial sums), slices added in order.
+__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int k_splits,
+                                     int64_t MN, __half* __restrict__ Y) {
+  const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i >= MN) return;
+  if ((MN & 3) == 0) {   // every slice's start is 16-byte aligned
+    float4 acc = *reinterpret_cast<const float4*>(partial + i);
+    for (int s = 1; s < k_splits; ++s) {
+      const float4 v = *reinterpret_cast<const float4*>(partial + static_cast<int64_t>(s) * MN + i);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    *reinterpret_cast<__half2*>(Y + i) = __floats2half2_rn(acc.x, acc.y);
+    *reinterpret_cast<__half2*>(Y + i + 2) = __floats2half2_rn(acc.z, acc.w);
+  } else {
+    for (int64_t e = i; e < MN; ++e) {
+      float acc = partial[e];
+      for (int s = 1; s < k_splits; ++s) acc += partial[static_cast<int64_t>(s) * MN + e];
+      Y[e] = __float2half_rn(acc);
+    }
   }
 }
 
