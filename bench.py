@@ -53,6 +53,13 @@ def peaks():
             "source": "fallback"}
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
+# the current kernels on these workloads: the three M = 1 decode launches of a step, averaged,
+# and the 4-bit M = 2048 [28672, 8192] prefill launch. Set to None when a kernel changes.
+DECODE_TRAFFIC_PER_LAUNCH = (8.825344e6 + 23.644672e6 + 23.658240e6) / 3
+PREFILL_TRAFFIC_PER_LAUNCH = 0.199680768e9 + 0.100501504e9
+
+
 def gemm_bytes(M, N, K, bits=4):
     return N * K * bits // 8 + N * (K // GROUP) * 3 + 2 * M * K + 2 * M * N
 
@@ -577,11 +584,16 @@ def run_b200(args, world, rank, local):
             "parallelism": f"replicas x{world} (no data-path collective)",
         },
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": pk["hbm_gbs"],
-                     "unit": "GB/s", "frac": per_gpu / pk["hbm_gbs"], "traffic": None,
-                     "kernel": "gemv_w4a16_kernel", "peak_source": pk["source"],
+                     "unit": "GB/s", "frac": per_gpu / pk["hbm_gbs"],
+                     "traffic": DECODE_TRAFFIC_PER_LAUNCH,
+                     "algorithmic_bytes_per_launch": step_bytes / len(synth.DECODE_SHAPES),
+                     "kernel": "gemv_stream_kernel<1, true>", "peak_source": pk["source"],
+                     "peak_kind": "measured copy bandwidth (burst)",
                      "frac_of_8TBps_nominal": per_gpu / 8000.0},
         "prefill": {"metric": "TFLOP/s at M=2048", "value": pf_value, "unit": "TFLOP/s",
                     "per_shape": prefill, "peak": pk["bf16_tflops"],
+                    "peak_kind": "measured bf16 cuBLAS burst (fp16 has the same dense rate)",
+                    "traffic_28672x8192": PREFILL_TRAFFIC_PER_LAUNCH,
                     "frac": pf_value / pk["bf16_tflops"] if prefill else None,
                     "kernel": "tc_gemm_kernel"},
         "sweep": sweep,

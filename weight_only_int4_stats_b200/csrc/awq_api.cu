@@ -116,9 +116,10 @@ awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_ro
   a.row_tiles = static_cast<int>((a_rows + awq::kTcBM - 1) / awq::kTcBM);
   a.rows_total = a_rows;
   if (a.k_splits < 1) a.k_splits = 1;
-  const int64_t blocks = static_cast<int64_t>(a.m_tiles) * a.row_tiles * a.k_splits;
-  if (blocks > 0x7FFFFFFFLL) return AWQ_ERR_INVALID_ARG;
-  kern<<<static_cast<unsigned>(blocks), awq::kTcThreads, L::kSmem, st>>>(tx, ta, a);
+  const int64_t units = static_cast<int64_t>(a.m_tiles) * a.row_tiles * a.k_splits;
+  const int64_t sms = num_sms();
+  const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);   // persistent
+  kern<<<grid, awq::kTcThreads, L::kSmem, st>>>(tx, ta, a);
   return launch_status();
 }
 
@@ -197,11 +198,10 @@ int splitk_for(int64_t M, int64_t N, int64_t K) {
   const int64_t bn = tc_bn_for(M);
   const int64_t tiles = ((N + awq::kTcBM - 1) / awq::kTcBM) * ((M + bn - 1) / bn);
   const int64_t sms = num_sms();
-  // CTAs of the wider tiles need more than half an SM's shared memory (one per SM); the
-  // split never adds a second wave of CTAs
-  const int64_t resident = sms * (bn <= 32 ? 2 : 1);
+  // the persistent kernel runs one CTA per SM: fill the SMs once, with about one work unit
+  // per SM (more would only queue behind each other)
   if (tiles >= sms) return 1;
-  int64_t s = resident / tiles;
+  int64_t s = sms / tiles;
   const int64_t by_groups = (K / awq::kGroup) / 2;
   const int64_t by_traffic = K / (8 * M);
   if (s > by_groups) s = by_groups;

@@ -8,18 +8,17 @@
 // Swap-AB formulation: the MMA's M side is 128 weight rows (output features n) and its N
 // side is BN tokens, so D = W_tile * X_tile^T lands in TMEM as 128 lanes (one per output
 // feature) x BN fp32 columns (one per token), and each dequantized weight is reused across
-// BN tokens. One CTA computes one 128 x BN tile with a 4-stage shared-memory ring of
-// 64-wide K slices:
-//   warp 0      TMA producer: X slice (128-byte swizzle) and the A source slice;
-//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer (kind::f16, fp32 acc);
-//   warps 2..5  A builders (packed source only): 16-byte packed chunks from shared memory
-//               -> fp16 (q - z) * scale in registers -> the canonical 128-byte swizzled
-//               K-major layout, then fence.proxy.async so the tensor core sees the writes;
-//               afterwards the same four warps run the epilogue (tcgen05.ld of their
-//               32-lane quarter of TMEM).
-// Epilogues: fp16 store of Y[m, n], or (search) each weight row's sum over the tile's
-// tokens of the squared output, written as one fp64 partial per (token tile, row).
-// Tiles are visited in a grouped order (see tile_of_block) for L2 reuse.
+// BN tokens. Persistent: one CTA per SM walks the (tile, K slice) work units in a grouped
+// order (see tile_of_block) with a shared-memory ring of 64-wide K stages that runs on
+// across tiles, and two TMEM accumulators so a tile's epilogue overlaps the next tile's
+// main loop:
+//   warp 0       TMA producer: X slice (128-byte swizzle) and the A source slice;
+//   warp 1       TMEM allocator and single-thread tcgen05.mma issuer (kind::f16, fp32 acc);
+//   warps 2..9   A builders (packed sources): 16-byte packed chunks from shared memory ->
+//                fp16 (q - z) * scale in registers -> the canonical 128-byte swizzled
+//                K-major layout, then fence.proxy.async so the tensor core sees the writes;
+//   warps 10..13 epilogue: tcgen05.ld of their 32-lane quarter of the finished accumulator,
+//                then fp16 Y, fp32 split-K partials, or (search) per-row sums of squares.
 // Every mbarrier wait is bounded; a timeout sets the device status word and the roles
 // leave their loops so the CTA still releases its TMEM and exits.
 #pragma once
@@ -29,9 +28,9 @@ namespace awq {
 
 constexpr int kTcBM = 128;      // weight rows per tile (MMA M)
 constexpr int kTcBK = 64;       // K per stage: one 128-byte swizzle atom of fp16
-constexpr int kTcStages = 4;
-constexpr int kTcBuilders = 8;  // A-builder / epilogue warps
-constexpr int kTcThreads = (2 + kTcBuilders) * 32;
+constexpr int kTcBuilders = 8;  // A-builder warps
+constexpr int kTcEpiWarps = 4;  // epilogue warps (one per TMEM lane quarter)
+constexpr int kTcThreads = (2 + kTcBuilders + kTcEpiWarps) * 32;
 constexpr int kTcPk3Slots = 2;  // 3-bit packed ring: one 128-k group (48 B per row) per slot
 
 enum class ASrc : int { kPacked4 = 0, kPacked3 = 1, kFp16 = 2 };
@@ -39,23 +38,23 @@ enum class Epi : int { kStoreY = 0, kRowSumSq = 1 };
 
 template <int BN, ASrc kA>
 struct TcLayout {
+  static constexpr int kStages = BN >= 256 ? 4 : 6;
   static constexpr int kXBytes = BN * kTcBK * 2;
   static constexpr int kABytes = kTcBM * kTcBK * 2;
   // packed source per stage (4-bit) or per ring slot (3-bit, one group of 128 k)
   static constexpr int kPBytes = kA == ASrc::kPacked4 ? kTcBM * kTcBK / 2
                                : kA == ASrc::kPacked3 ? kTcBM * 48 : 0;
-  static constexpr int kPSlots = kA == ASrc::kPacked3 ? kTcPk3Slots : kTcStages;
+  static constexpr int kPSlots = kA == ASrc::kPacked3 ? kTcPk3Slots : kStages;
   static constexpr int kXOff = 0;
-  static constexpr int kAOff = kXOff + kTcStages * kXBytes;
-  static constexpr int kPOff = kAOff + kTcStages * kABytes;
-  static constexpr int kRedOff = kPOff + kPSlots * kPBytes;          // 128 doubles
-  static constexpr int kBarOff = kRedOff + kTcBM * 8;
-  // full[S], empty[S], built[S], pfull[2], pempty[2], acc_full, tmem slot
-  static constexpr int kBytes = kBarOff + (3 * kTcStages + 2 * kTcPk3Slots + 1) * 8 + 16;
+  static constexpr int kAOff = kXOff + kStages * kXBytes;
+  static constexpr int kPOff = kAOff + kStages * kABytes;
+  static constexpr int kBarOff = kPOff + kPSlots * kPBytes;
+  // full[S], empty[S], built[S], pfull[2], pempty[2], acc_full[2], acc_empty[2], tmem slot
+  static constexpr int kBytes = kBarOff + (3 * kStages + 2 * kTcPk3Slots + 4) * 8 + 16;
   static constexpr int kSmem = kBytes + 1024;   // slack for 1024-byte alignment
   static constexpr uint32_t kTxBytes =
       kXBytes + (kA == ASrc::kFp16 ? kABytes : kA == ASrc::kPacked4 ? kPBytes : 0);
-  static constexpr uint32_t kTmemCols = BN;     // fp32 accumulator columns (power of 2)
+  static constexpr uint32_t kTmemCols = 2 * BN;   // two fp32 accumulators (power of 2)
 };
 
 struct TcArgs {
@@ -70,13 +69,13 @@ struct TcArgs {
   int m_tiles;
   int row_tiles;        // 128-row tiles of the A matrix
   int64_t rows_total;   // rows of the A matrix (row_tiles * 128 for the search)
-  int k_splits;         // > 1: each CTA covers a group-aligned slice of K (split-K)
+  int k_splits;         // > 1: each work unit covers a group-aligned slice of K (split-K)
   float* partial;       // [k_splits, M, N] fp32 partial sums (split-K store epilogue)
 };
 
-// Grouped tile order: consecutive CTAs sweep the token tiles of a group of kTcRasterRows
-// weight-row tiles, so the CTAs resident at one time share a few A tiles and a few X tiles
-// in L2 instead of each streaming its own X tile from HBM.
+// Grouped tile order: consecutive work units sweep the token tiles of a group of
+// kTcRasterRows weight-row tiles, so the units in flight at one time share a few A tiles and
+// a few X tiles in L2 instead of each streaming its own X tile from HBM.
 constexpr int kTcRasterRows = 16;
 
 __device__ __forceinline__ void tile_of_block(int64_t bid, int row_tiles, int m_tiles,
@@ -88,6 +87,23 @@ __device__ __forceinline__ void tile_of_block(int64_t bid, int row_tiles, int m_
   const int rows_here = row_tiles - first < kTcRasterRows ? row_tiles - first : kTcRasterRows;
   row_tile = first + static_cast<int>(in_group % rows_here);
   m_tile = static_cast<int>(in_group / rows_here);
+}
+
+struct TcUnit {
+  int row_tile, m_tile, ksplit, kb0, nkb;
+};
+
+__device__ __forceinline__ TcUnit unit_of(int64_t u, const TcArgs& a) {
+  TcUnit t;
+  const int64_t tiles = static_cast<int64_t>(a.row_tiles) * a.m_tiles;
+  t.ksplit = static_cast<int>(u / tiles);
+  tile_of_block(u % tiles, a.row_tiles, a.m_tiles, t.row_tile, t.m_tile);
+  const int G = static_cast<int>(a.K / kGroup);
+  const int kb0 = 2 * static_cast<int>(static_cast<int64_t>(t.ksplit) * G / a.k_splits);
+  const int kb1 = 2 * static_cast<int>(static_cast<int64_t>(t.ksplit + 1) * G / a.k_splits);
+  t.kb0 = kb0;
+  t.nkb = kb1 - kb0;
+  return t;
 }
 
 // Dequantize one 4-bit packed word (8 consecutive k) to four fp16 pairs (q - z) * sc.
@@ -136,44 +152,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                    const __grid_constant__ CUtensorMap tmap_a, const TcArgs args) {
   using L = TcLayout<BN, kA>;
+  constexpr int S = L::kStages;
   constexpr bool kPacked = kA != ASrc::kFp16;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* empty = full + kTcStages;
-  uint64_t* built = empty + kTcStages;
-  uint64_t* pfull = built + kTcStages;
+  uint64_t* empty = full + S;
+  uint64_t* built = empty + S;
+  uint64_t* pfull = built + S;
   uint64_t* pempty = pfull + kTcPk3Slots;
   uint64_t* acc_full = pempty + kTcPk3Slots;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
-  double* red = reinterpret_cast<double*>(smem + L::kRedOff);
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  int m_tile, row_tile;
-  const int64_t tiles = static_cast<int64_t>(args.row_tiles) * args.m_tiles;
-  const int ksplit = static_cast<int>(blockIdx.x / tiles);
-  tile_of_block(blockIdx.x % tiles, args.row_tiles, args.m_tiles, row_tile, m_tile);
-  const int64_t m0 = static_cast<int64_t>(m_tile) * BN;
-  const int64_t row0 = static_cast<int64_t>(row_tile) * kTcBM;   // row in the A matrix
-  // this CTA's K slice, in whole groups of 128 (two 64-wide stages per group)
-  const int G = static_cast<int>(args.K / kGroup);
-  const int kb0 = 2 * static_cast<int>(static_cast<int64_t>(ksplit) * G / args.k_splits);
-  const int kb1 = 2 * static_cast<int>(static_cast<int64_t>(ksplit + 1) * G / args.k_splits);
-  const int nkb = kb1 - kb0;
+  const int64_t units =
+      static_cast<int64_t>(args.row_tiles) * args.m_tiles * args.k_splits;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-      mbar_init(&built[s], kTcBuilders * 32);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&built[i], kTcBuilders * 32);
     }
-    for (int s = 0; s < kTcPk3Slots; ++s) {
-      mbar_init(&pfull[s], 1);
-      mbar_init(&pempty[s], kTcBuilders * 32);
+    for (int i = 0; i < kTcPk3Slots; ++i) {
+      mbar_init(&pfull[i], 1);
+      mbar_init(&pempty[i], kTcBuilders * 32);
     }
-    mbar_init(acc_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], kTcEpiWarps * 32);
+    }
     fence_barrier_init();
     tma_prefetch_desc(&tmap_x);
     tma_prefetch_desc(&tmap_a);
@@ -185,133 +196,169 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_d = *tmem_slot;
+  const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      for (int i = 0; i < nkb; ++i) {
-        const int kb = kb0 + i;
-        const int s = i % kTcStages;
-        const uint32_t ph = (i / kTcStages) & 1;
-        if (kA == ASrc::kPacked3 && (i & 1) == 0) {
-          const int li = i >> 1, ps = li % kTcPk3Slots;
-          if (!mbar_wait(&pempty[ps], ((li / kTcPk3Slots) & 1) ^ 1)) break;
-          mbar_arrive_expect_tx(&pfull[ps], L::kPBytes);
-          tma_load_2d(smem + L::kPOff + ps * L::kPBytes, &tmap_a, &pfull[ps], (kb >> 1) * 12,
-                      static_cast<int32_t>(row0));
+      int64_t it = 0, pit = 0;   // stage and 3-bit pair counters, continuous across units
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const TcUnit t = unit_of(u, args);
+        const int64_t m0 = static_cast<int64_t>(t.m_tile) * BN;
+        const int64_t row0 = static_cast<int64_t>(t.row_tile) * kTcBM;
+        for (int i = 0; i < t.nkb; ++i, ++it) {
+          const int kb = t.kb0 + i;
+          const int s = static_cast<int>(it % S);
+          const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+          if (kA == ASrc::kPacked3 && (i & 1) == 0) {
+            const int ps = static_cast<int>(pit % kTcPk3Slots);
+            if (!mbar_wait(&pempty[ps], static_cast<uint32_t>((pit / kTcPk3Slots) & 1) ^ 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&pfull[ps], L::kPBytes);
+            tma_load_2d(smem + L::kPOff + ps * L::kPBytes, &tmap_a, &pfull[ps], (kb >> 1) * 12,
+                        static_cast<int32_t>(row0));
+            ++pit;
+          }
+          if (!mbar_wait(&empty[s], ph ^ 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], L::kTxBytes);
+          tma_load_2d(smem + L::kXOff + s * L::kXBytes, &tmap_x, &full[s], kb * kTcBK,
+                      static_cast<int32_t>(m0));
+          if (kA == ASrc::kFp16)
+            tma_load_2d(smem + L::kAOff + s * L::kABytes, &tmap_a, &full[s], kb * kTcBK,
+                        static_cast<int32_t>(row0));
+          else if (kA == ASrc::kPacked4)
+            tma_load_2d(smem + L::kPOff + s * L::kPBytes, &tmap_a, &full[s], kb * (kTcBK / 8),
+                        static_cast<int32_t>(row0));
         }
-        if (!mbar_wait(&empty[s], ph ^ 1)) break;
-        mbar_arrive_expect_tx(&full[s], L::kTxBytes);
-        tma_load_2d(smem + L::kXOff + s * L::kXBytes, &tmap_x, &full[s], kb * kTcBK,
-                    static_cast<int32_t>(m0));
-        if (kA == ASrc::kFp16)
-          tma_load_2d(smem + L::kAOff + s * L::kABytes, &tmap_a, &full[s], kb * kTcBK,
-                      static_cast<int32_t>(row0));
-        else if (kA == ASrc::kPacked4)
-          tma_load_2d(smem + L::kPOff + s * L::kPBytes, &tmap_a, &full[s], kb * (kTcBK / 8),
-                      static_cast<int32_t>(row0));
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = f16_idesc(kTcBM, BN);
+      int64_t it = 0, lt = 0;
       bool ok = true;
-      for (int i = 0; i < nkb && ok; ++i) {
-        const int s = i % kTcStages;
-        const uint32_t ph = (i / kTcStages) & 1;
-        ok = mbar_wait(&full[s], ph);
-        if (ok && kPacked) ok = mbar_wait(&built[s], ph);
-        if (!ok) break;
+      for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x, ++lt) {
+        const TcUnit t = unit_of(u, args);
+        const int buf = static_cast<int>(lt & 1);
+        const uint32_t acc_ph = static_cast<uint32_t>((lt >> 1) & 1);
+        if (!mbar_wait(&acc_empty[buf], acc_ph ^ 1)) break;   // epilogue released the buffer
         tc_fence_after();
-        const uint32_t a_base = smem_u32(smem + L::kAOff + s * L::kABytes);
-        const uint32_t x_base = smem_u32(smem + L::kXOff + s * L::kXBytes);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+        for (int i = 0; i < t.nkb; ++i, ++it) {
+          const int s = static_cast<int>(it % S);
+          const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+          ok = mbar_wait(&full[s], ph);
+          if (ok && kPacked) ok = mbar_wait(&built[s], ph);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + L::kAOff + s * L::kABytes);
+          const uint32_t x_base = smem_u32(smem + L::kXOff + s * L::kXBytes);
 #pragma unroll
-        for (int kk = 0; kk < kTcBK / 16; ++kk) {
-          tc_mma_f16(tmem_d, sw128_kmajor_desc(a_base + kk * 32),
-                     sw128_kmajor_desc(x_base + kk * 32), idesc, (i | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < kTcBK / 16; ++kk) {
+            tc_mma_f16(d_tmem, sw128_kmajor_desc(a_base + kk * 32),
+                       sw128_kmajor_desc(x_base + kk * 32), idesc, (i | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
         }
-        tc_commit(&empty[s]);
+        tc_commit(&acc_full[buf]);
       }
-      tc_commit(acc_full);
+    }
+  } else if (warp < 2 + kTcBuilders) {
+    // ------------------------------------------------------------------ A builders
+    if (kPacked) {
+      const int t = threadIdx.x - 64;          // 0..255
+      const int r = t >> 1, h = t & 1;         // tile row, 32-k half of the 64-k stage
+      const int64_t N = args.N;
+      int64_t it = 0, pit = 0;
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const TcUnit tu = unit_of(u, args);
+        const int64_t n = static_cast<int64_t>(tu.row_tile) * kTcBM + r;
+        __half2 lo, hi, sc;
+        for (int i = 0; i < tu.nkb; ++i, ++it) {
+          const int kb = tu.kb0 + i;
+          const int s = static_cast<int>(it % S);
+          const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+          if ((i & 1) == 0) {    // new group of 128: this row's zero point and scale
+            const int64_t g = kb >> 1;
+            const uint32_t z = n < N ? args.zeros[g * N + n] : 0u;
+            const __half sv = n < N ? args.scales[g * N + n] : __float2half(0.0f);
+            lo = u32_as_h2((0x6400u | z) * 0x00010001u);
+            hi = u32_as_h2((0xD400u | (z << 4)) * 0x00010001u);
+            sc = __half2half2(sv);
+          }
+          bool got = mbar_wait(&full[s], ph) && mbar_wait(&empty[s], ph ^ 1);
+          const int ps = static_cast<int>(pit % kTcPk3Slots);
+          if (kA == ASrc::kPacked3 && got)
+            got = mbar_wait(&pfull[ps], static_cast<uint32_t>((pit / kTcPk3Slots) & 1));
+          ok = __all_sync(0xffffffffu, got);   // keep the warp converged for .aligned ops
+          if (!ok) break;
+          uint8_t* atile = smem + L::kAOff + s * L::kABytes;
+          if (kA == ASrc::kPacked4) {
+            const uint8_t* ptile = smem + L::kPOff + s * L::kPBytes;
+            const uint4 pw = *reinterpret_cast<const uint4*>(ptile + t * 16);   // row r, half h
+            const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 o = dequant_word_scaled(words[q], lo, hi, sc);
+              *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + q)) = o;
+            }
+          } else {
+            const uint32_t* pw = reinterpret_cast<const uint32_t*>(
+                smem + L::kPOff + ps * L::kPBytes + r * 48 + 12 * (2 * (i & 1) + h));
+            const uint32_t w0 = pw[0], w1 = pw[1], w2 = pw[2];
+            uint4 o;
+#define AWQ_DQ3_CHUNK(I)                                                   \
+  o.x = dequant3_pair<I, 0>(w0, w1, w2, lo, sc);                          \
+  o.y = dequant3_pair<I, 1>(w0, w1, w2, lo, sc);                          \
+  o.z = dequant3_pair<I, 2>(w0, w1, w2, lo, sc);                          \
+  o.w = dequant3_pair<I, 3>(w0, w1, w2, lo, sc);                          \
+  *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + I)) = o;
+            AWQ_DQ3_CHUNK(0)
+            AWQ_DQ3_CHUNK(1)
+            AWQ_DQ3_CHUNK(2)
+            AWQ_DQ3_CHUNK(3)
+#undef AWQ_DQ3_CHUNK
+            if (i & 1) {                      // both stages of the group are built
+              mbar_arrive(&pempty[ps]);
+              ++pit;
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&built[s]);
+        }
+      }
     }
   } else {
-    // ------------------------------------------------------------------ A builders
-    const int t = threadIdx.x - 64;            // 0..255
-    const int r = t >> 1, h = t & 1;           // tile row, 32-k half of the 64-k stage
-    const int64_t n = row0 + r;
-    const int64_t N = args.N;
-    bool ok = true;
-    if (kPacked) {
-      __half2 lo, hi, sc;
-      for (int i = 0; i < nkb; ++i) {
-        const int kb = kb0 + i;
-        const int s = i % kTcStages;
-        const uint32_t ph = (i / kTcStages) & 1;
-        if ((i & 1) == 0) {    // new group of 128: this row's zero point and scale
-          const int64_t g = kb >> 1;
-          const uint32_t z = n < N ? args.zeros[g * N + n] : 0u;
-          const __half sv = n < N ? args.scales[g * N + n] : __float2half(0.0f);
-          lo = u32_as_h2((0x6400u | z) * 0x00010001u);
-          hi = __hneg2(u32_as_h2((0x5400u | (z << 4)) * 0x00010001u));
-          sc = __half2half2(sv);
-        }
-        bool got = mbar_wait(&full[s], ph) && mbar_wait(&empty[s], ph ^ 1);
-        const int li = i >> 1, ps = li % kTcPk3Slots;
-        if (kA == ASrc::kPacked3 && got) got = mbar_wait(&pfull[ps], (li / kTcPk3Slots) & 1);
-        ok = __all_sync(0xffffffffu, got);   // keep the warp converged for .aligned ops
-        if (!ok) break;
-        uint8_t* atile = smem + L::kAOff + s * L::kABytes;
-        if (kA == ASrc::kPacked4) {
-          const uint8_t* ptile = smem + L::kPOff + s * L::kPBytes;
-          const uint4 pw = *reinterpret_cast<const uint4*>(ptile + t * 16);   // row r, half h
-          const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 o = dequant_word_scaled(words[i], lo, hi, sc);
-            *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + i)) = o;
-          }
-        } else {
-          const uint32_t* pw = reinterpret_cast<const uint32_t*>(
-              smem + L::kPOff + ps * L::kPBytes + r * 48 + 12 * (2 * (i & 1) + h));
-          const uint32_t w0 = pw[0], w1 = pw[1], w2s = pw[2];
-          uint4 o;
-#define AWQ_DQ3_CHUNK(I)                                                   \
-  o.x = dequant3_pair<I, 0>(w0, w1, w2s, lo, sc);                         \
-  o.y = dequant3_pair<I, 1>(w0, w1, w2s, lo, sc);                         \
-  o.z = dequant3_pair<I, 2>(w0, w1, w2s, lo, sc);                         \
-  o.w = dequant3_pair<I, 3>(w0, w1, w2s, lo, sc);                         \
-  *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + I)) = o;
-          AWQ_DQ3_CHUNK(0)
-          AWQ_DQ3_CHUNK(1)
-          AWQ_DQ3_CHUNK(2)
-          AWQ_DQ3_CHUNK(3)
-#undef AWQ_DQ3_CHUNK
-          if (i & 1) mbar_arrive(&pempty[ps]);    // both stages of the group are built
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&built[s]);
-      }
-    }
     // ------------------------------------------------------------------ epilogue
-    // Warp w reads TMEM lane quarter (w % 4) -- the only one it may access -- and half of
-    // the BN token columns; the two halves of a row's sum of squares meet in shared memory.
-    if (ok) ok = mbar_wait(acc_full, 0);
-    ok = __all_sync(0xffffffffu, ok);
+    // Warp w reads TMEM lane quarter (w % 4), the only one it may access: 32 weight rows of
+    // the finished accumulator, all BN token columns.
     const int wq = warp & 3;
-    const int half = (warp - 2) >> 2;
     const int row = 32 * wq + lane;
-    const int64_t arow = row0 + row;
-    double sumsq = 0.0;
-    if (ok) {
+    int64_t lt = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x, ++lt) {
+      const TcUnit t = unit_of(u, args);
+      const int buf = static_cast<int>(lt & 1);
+      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], static_cast<uint32_t>((lt >> 1) & 1)));
+      if (!ok) break;
       tc_fence_after();
-      constexpr int kHalf = BN / 2;
+      const int64_t m0 = static_cast<int64_t>(t.m_tile) * BN;
+      const int64_t arow = static_cast<int64_t>(t.row_tile) * kTcBM + row;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * wq) << 16) +
+                             static_cast<uint32_t>(buf * BN);
+      double sumsq = 0.0;
 #pragma unroll 1
-      for (int cb = 0; cb < kHalf; cb += 16) {
+      for (int col = 0; col < BN; col += 16) {
         uint32_t v[16];
-        const int col = half * kHalf + cb;
-        tmem_ld_32x32b_x16(tmem_d + (static_cast<uint32_t>(32 * wq) << 16) + col, v);
+        tmem_ld_32x32b_x16(taddr + col, v);
         tmem_ld_wait();
         if (kEpi == Epi::kStoreY) {
           if (arow < args.N) {
@@ -322,7 +369,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (m < args.M) args.Y[m * args.N + arow] = __float2half_rn(__uint_as_float(v[j]));
               }
             } else {
-              float* P = args.partial + static_cast<int64_t>(ksplit) * args.M * args.N;
+              float* P = args.partial + static_cast<int64_t>(t.ksplit) * args.M * args.N;
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
                 const int64_t m = m0 + col + j;
@@ -340,12 +387,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           sumsq += static_cast<double>(part);
         }
       }
-    }
-    if (kEpi == Epi::kRowSumSq) {
-      if (half == 1) red[row] = sumsq;
-      named_bar_sync(1, kTcBuilders * 32);
-      if (half == 0 && ok)
-        args.row_part[static_cast<int64_t>(m_tile) * args.rows_total + arow] = sumsq + red[row];
+      if (kEpi == Epi::kRowSumSq)
+        args.row_part[static_cast<int64_t>(t.m_tile) * args.rows_total + arow] = sumsq;
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);            // the MMA may overwrite this accumulator
     }
   }
 
@@ -353,7 +398,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_d, L::kTmemCols);
+    tmem_dealloc(tmem_base, L::kTmemCols);
   }
 }
 

@@ -88,18 +88,19 @@ __device__ __forceinline__ QuantGroup group_params(const float (&w)[16]) {
   return g;
 }
 
-// q = clamp(rint(w' / sc) + z, 0, qmax) with the IEEE quotient. rint of the correctly rounded
-// quotient can only differ from rint of a nearby value where the two straddle a half-integer,
-// so the product w' * rcp (within 2^-22 relative of the exact quotient) decides the code
-// unless it lies within a safe margin of a half-integer; only then is the quotient formed
-// with an IEEE division.
+// q = clamp(rint(w' / sc) + z, 0, qmax) with the IEEE quotient. The product t = w' * rcp,
+// rcp = 1/sc correctly rounded, is within 2^-23 |w'/sc| (two roundings) of the exact
+// quotient, and rint of the correctly rounded quotient can only differ from rint(t) where
+// the two straddle a half-integer. So for |t| <= 32 (absolute error <= 2^-18) rint(t) is the
+// code unless t lies within 2^-17 of a half-integer; only then is the quotient formed with
+// an IEEE division. For |t| > 32 the code clamps to 0 or qmax whatever the rounding, since
+// 0 <= z <= 15.
 template <int kBits>
 __device__ __forceinline__ float code_of(float wp, const QuantGroup& g) {
   constexpr float qmax = static_cast<float>((1 << kBits) - 1);
   const float t = __fmul_rn(wp, g.rcp);
   float r = rintf(t);
-  const float gap = fabsf(fabsf(__fsub_rn(t, r)) - 0.5f);
-  if (gap <= fmaxf(fabsf(t), 1.0f) * 0x1p-18f) r = rintf(__fdiv_rn(wp, g.sc));
+  if (fabsf(__fsub_rn(t, r)) >= 0.5f - 0x1p-17f) r = rintf(__fdiv_rn(wp, g.sc));
   return fminf(fmaxf(__fadd_rn(r, g.z), 0.0f), qmax);
 }
 
