@@ -57,7 +57,7 @@ def peaks():
 # the current kernels on these workloads: the three M = 1 decode launches of a step, averaged,
 # and the 4-bit M = 2048 [28672, 8192] prefill launch. Set to None when a kernel changes.
 DECODE_TRAFFIC_PER_LAUNCH = (8.825344e6 + 23.644672e6 + 23.658240e6) / 3
-PREFILL_TRAFFIC_PER_LAUNCH = 0.199680768e9 + 0.100501504e9
+PREFILL_TRAFFIC_PER_LAUNCH = None   # tensor-core GEMM changed since its last capture
 
 
 def gemm_bytes(M, N, K, bits=4):

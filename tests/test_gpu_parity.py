@@ -180,6 +180,17 @@ def test_gemm_split_k_ragged(awq, M, N, K, bits):
     _check_gemm(awq, X, qw, sc, z, N, K, bits)
 
 
+@pytest.mark.parametrize("bits", [4, 3])
+@pytest.mark.parametrize("M,N,K", [(40, 512, 2304), (20, 640, 1152), (96, 256, 1664),
+                                   (250, 384, 640)])
+def test_gemm_group_slots_ragged(awq, M, N, K, bits):
+    # N % 16 == 0, so scales and zero points travel by TMA with the packed codes, several
+    # groups per load; K slices (split-K) and K itself end inside a multi-group load
+    W, X, m = rand_layer(3 * M + N + K + bits, N, K, M)
+    qw, sc, z = _packed(W, np.sqrt(m).astype(np.float32), bits)
+    _check_gemm(awq, X, qw, sc, z, N, K, bits)
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_gemm_3bit_decode_sizes(awq, M):
     N, K = 320, 768

@@ -102,16 +102,29 @@ awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_ro
     if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a_rows, args.K, awq::kTcBM,
                       awq::kTcBK, true))
       return AWQ_ERR_CUDA;
-  } else if (kA == ASrc::kPacked4) {
+  } else if (kA == ASrc::kPacked4) {   // kPG groups of 16 words (64 bytes) per row per load
     if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a_rows, args.K / 8,
-                      awq::kTcBM, awq::kTcBK / 8, false))
+                      awq::kTcBM, L::kPRowBytes / 4, false))
       return AWQ_ERR_CUDA;
-  } else {   // 3-bit: one 128-k group = 12 words (48 bytes) per row per load
+  } else {   // 3-bit: kPG groups of 12 words (48 bytes) per row per load
     if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a_rows, 3 * args.K / 32,
-                      awq::kTcBM, 12, false))
+                      awq::kTcBM, L::kPRowBytes / 4, false))
       return AWQ_ERR_CUDA;
   }
+  // scales [G, N] fp16 and zeros [G, N] u8 as TMA tiles of kPG groups x 128 rows, when the
+  // row stride of the zeros (N bytes) meets the 16-byte rule; otherwise the maps go unused
+  CUtensorMap ts = ta, tz = ta;
   awq::TcArgs a = args;
+  a.sz_tma = 0;
+  if (kA != ASrc::kFp16 && args.N % 16 == 0) {
+    const int64_t G = args.K / awq::kGroup;
+    if (!make_tmap_2d(&ts, args.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, G, args.N, L::kPG,
+                      awq::kTcBM, false) ||
+        !make_tmap_2d(&tz, args.zeros, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, G, args.N, L::kPG,
+                      awq::kTcBM, false))
+      return AWQ_ERR_CUDA;
+    a.sz_tma = 1;
+  }
   a.m_tiles = static_cast<int>((M + BN - 1) / BN);
   a.row_tiles = static_cast<int>((a_rows + awq::kTcBM - 1) / awq::kTcBM);
   a.rows_total = a_rows;
@@ -119,7 +132,7 @@ awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_ro
   const int64_t units = static_cast<int64_t>(a.m_tiles) * a.row_tiles * a.k_splits;
   const int64_t sms = num_sms();
   const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);   // persistent
-  kern<<<grid, awq::kTcThreads, L::kSmem, st>>>(tx, ta, a);
+  kern<<<grid, awq::kTcThreads, L::kSmem, st>>>(tx, ta, ts, tz, a);
   return launch_status();
 }
 

@@ -12,13 +12,26 @@
 // order (see tile_of_block) with a shared-memory ring of 64-wide K stages that runs on
 // across tiles, and two TMEM accumulators so a tile's epilogue overlaps the next tile's
 // main loop:
-//   warp 0       TMA producer: X slice (128-byte swizzle) and the A source slice;
+//   warp 5       TMA producer: X slice (128-byte swizzle), and the A slice (fp16 source);
 //   warp 1       TMEM allocator and single-thread tcgen05.mma issuer (kind::f16, fp32 acc);
-//   warps 2..9   A builders (packed sources): 16-byte packed chunks from shared memory ->
+//   warp 9       TMA producer of the packed source: kPG consecutive 128-k groups of packed
+//                weights (with their scales and zero points) per slot of a ring as deep as
+//                shared memory allows, running ahead of the stage ring. When few tokens share
+//                each weight the kernel streams weights from DRAM, and TMA tiles of 128 rows
+//                only reach full DRAM throughput with long rows (about 2.7 TB/s at 64 bytes
+//                per row, 4.7 at 128, 5.5-5.9 at 256 on B200), so narrow token tiles take
+//                four groups (256 bytes of 4-bit codes) per row per slot;
+//   warps 0, 2, 3, 4, 6, 7, 8, 10
+//                A builders (packed sources): 16-byte packed chunks from shared memory ->
 //                fp16 (q - z) * scale in registers -> the canonical 128-byte swizzled
 //                K-major layout, then fence.proxy.async so the tensor core sees the writes;
-//   warps 10..13 epilogue: tcgen05.ld of their 32-lane quarter of the finished accumulator,
-//                then fp16 Y, fp32 split-K partials, or (search) per-row sums of squares.
+//   warps 12..15 epilogue: tcgen05.ld of their 32-lane quarter of the finished accumulator,
+//                then fp16 Y, fp32 split-K partials, or (search) per-row sums of squares;
+//   warp 11      idle.
+// Warp w issues from sub-partition w % 4. The MMA issuer and both TMA producers share
+// sub-partition 1 and no builder runs there: a builder warp placed beside the MMA issuer
+// (or beside the X producer) was measured finishing its part of each stage 2000-3700
+// cycles after the other builders, which held every MMA back by as much.
 // Every mbarrier wait is bounded; a timeout sets the device status word and the roles
 // leave their loops so the CTA still releases its TMEM and exits.
 #pragma once
@@ -30,30 +43,47 @@ constexpr int kTcBM = 128;      // weight rows per tile (MMA M)
 constexpr int kTcBK = 64;       // K per stage: one 128-byte swizzle atom of fp16
 constexpr int kTcBuilders = 8;  // A-builder warps
 constexpr int kTcEpiWarps = 4;  // epilogue warps (one per TMEM lane quarter)
-constexpr int kTcThreads = (2 + kTcBuilders + kTcEpiWarps) * 32;
-constexpr int kTcPk3Slots = 2;  // 3-bit packed ring: one 128-k group (48 B per row) per slot
+constexpr int kTcThreads = 16 * 32;
+constexpr int kTcMmaWarp = 1;
+constexpr int kTcXWarp = 5;
+constexpr int kTcPackWarp = 9;
+constexpr int kTcIdleWarp = 11;
+constexpr int kTcEpiWarp0 = 12;   // warps 12..15: TMEM lane quarters 0..3 (warp % 4)
+constexpr int kTcPkSlotsMax = 16;   // deepest packed ring
+constexpr int kTcSmemMax = 232448;  // dynamic shared memory per CTA on sm_100
 
 enum class ASrc : int { kPacked4 = 0, kPacked3 = 1, kFp16 = 2 };
 enum class Epi : int { kStoreY = 0, kRowSumSq = 1 };
 
 template <int BN, ASrc kA>
 struct TcLayout {
-  static constexpr int kStages = BN >= 256 ? 4 : 6;
+  static constexpr bool kPk = kA != ASrc::kFp16;
+  static constexpr int kStages = !kPk ? (BN >= 256 ? 4 : 6) : (BN >= 256 ? 4 : BN >= 64 ? 5 : 6);
   static constexpr int kXBytes = BN * kTcBK * 2;
   static constexpr int kABytes = kTcBM * kTcBK * 2;
-  // packed source per stage (4-bit) or per ring slot (3-bit, one group of 128 k)
-  static constexpr int kPBytes = kA == ASrc::kPacked4 ? kTcBM * kTcBK / 2
-                               : kA == ASrc::kPacked3 ? kTcBM * 48 : 0;
-  static constexpr int kPSlots = kA == ASrc::kPacked3 ? kTcPk3Slots : kStages;
+  // packed source: kPG groups (2 kPG stages) per ring slot
+  static constexpr int kPG = !kPk ? 1 : BN <= 64 ? 4 : BN <= 128 ? 2 : 1;
+  static constexpr int kPGroupBytes = kA == ASrc::kPacked4 ? 64 : kA == ASrc::kPacked3 ? 48 : 0;
+  static constexpr int kPRowBytes = kPG * kPGroupBytes;
+  static constexpr int kPBytes = kTcBM * kPRowBytes;
+  // the slot's fp16 scales [kPG][128] then its zero points [kPG][128]
+  static constexpr int kSZBytes = kPG * (kTcBM * 2 + kTcBM);
+  // as many packed slots as the shared memory left by the stages holds (1024 bytes of
+  // alignment slack and 512 of barriers reserved)
+  static constexpr int kPFit =
+      (kTcSmemMax - 1024 - 512 - kStages * (kXBytes + kABytes)) / (kPBytes + kSZBytes);
+  static constexpr int kPSlots =
+      kA == ASrc::kFp16 ? 0 : (kPFit < kTcPkSlotsMax ? kPFit : kTcPkSlotsMax);
+  static constexpr int kPBars = kPSlots > 0 ? kPSlots : 1;   // barrier pairs of the ring
   static constexpr int kXOff = 0;
   static constexpr int kAOff = kXOff + kStages * kXBytes;
   static constexpr int kPOff = kAOff + kStages * kABytes;
-  static constexpr int kBarOff = kPOff + kPSlots * kPBytes;
-  // full[S], empty[S], built[S], pfull[2], pempty[2], acc_full[2], acc_empty[2], tmem slot
-  static constexpr int kBytes = kBarOff + (3 * kStages + 2 * kTcPk3Slots + 4) * 8 + 16;
+  static constexpr int kSZOff = kPOff + kPSlots * kPBytes;
+  static constexpr int kBarOff = kSZOff + kPSlots * kSZBytes;
+  // full[S], empty[S], built[S], pfull[P], pempty[P], acc_full[2], acc_empty[2], tmem slot
+  static constexpr int kBytes = kBarOff + (3 * kStages + 2 * kPBars + 4) * 8 + 16;
   static constexpr int kSmem = kBytes + 1024;   // slack for 1024-byte alignment
-  static constexpr uint32_t kTxBytes =
-      kXBytes + (kA == ASrc::kFp16 ? kABytes : kA == ASrc::kPacked4 ? kPBytes : 0);
+  static constexpr uint32_t kTxBytes = kXBytes + (kA == ASrc::kFp16 ? kABytes : 0);
   static constexpr uint32_t kTmemCols = 2 * BN;   // two fp32 accumulators (power of 2)
 };
 
@@ -71,6 +101,8 @@ struct TcArgs {
   int64_t rows_total;   // rows of the A matrix (row_tiles * 128 for the search)
   int k_splits;         // > 1: each work unit covers a group-aligned slice of K (split-K)
   float* partial;       // [k_splits, M, N] fp32 partial sums (split-K store epilogue)
+  int sz_tma;           // packed source: scales and zeros arrive by TMA with the packed group
+                        // (needs N % 16 == 0); else the builders load them from global memory
 };
 
 // Grouped tile order: consecutive work units sweep the token tiles of a group of
@@ -150,7 +182,9 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
 template <int BN, ASrc kA, Epi kEpi>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                   const __grid_constant__ CUtensorMap tmap_a, const TcArgs args) {
+                   const __grid_constant__ CUtensorMap tmap_a,
+                   const __grid_constant__ CUtensorMap tmap_s,
+                   const __grid_constant__ CUtensorMap tmap_z, const TcArgs args) {
   using L = TcLayout<BN, kA>;
   constexpr int S = L::kStages;
   constexpr bool kPacked = kA != ASrc::kFp16;
@@ -161,8 +195,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* empty = full + S;
   uint64_t* built = empty + S;
   uint64_t* pfull = built + S;
-  uint64_t* pempty = pfull + kTcPk3Slots;
-  uint64_t* acc_full = pempty + kTcPk3Slots;
+  constexpr int P = L::kPBars;
+  static_assert(!kPacked || L::kPSlots >= 2, "packed ring needs two slots");
+  static_assert(L::kSmem <= kTcSmemMax, "shared memory layout too large");
+  uint64_t* pempty = pfull + P;
+  uint64_t* acc_full = pempty + P;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
@@ -177,7 +214,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&empty[i], 1);
       mbar_init(&built[i], kTcBuilders * 32);
     }
-    for (int i = 0; i < kTcPk3Slots; ++i) {
+    for (int i = 0; i < P; ++i) {
       mbar_init(&pfull[i], 1);
       mbar_init(&pempty[i], kTcBuilders * 32);
     }
@@ -188,8 +225,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmap_x);
     tma_prefetch_desc(&tmap_a);
+    if (kPacked && args.sz_tma) {
+      tma_prefetch_desc(&tmap_s);
+      tma_prefetch_desc(&tmap_z);
+    }
   }
-  if (warp == 1) {
+  if (warp == kTcMmaWarp) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
@@ -198,10 +239,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == kTcXWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int64_t it = 0, pit = 0;   // stage and 3-bit pair counters, continuous across units
+      int64_t it = 0;   // stage counter, continuous across units
       bool ok = true;
       for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const TcUnit t = unit_of(u, args);
@@ -211,17 +252,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int kb = t.kb0 + i;
           const int s = static_cast<int>(it % S);
           const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-          if (kA == ASrc::kPacked3 && (i & 1) == 0) {
-            const int ps = static_cast<int>(pit % kTcPk3Slots);
-            if (!mbar_wait(&pempty[ps], static_cast<uint32_t>((pit / kTcPk3Slots) & 1) ^ 1)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&pfull[ps], L::kPBytes);
-            tma_load_2d(smem + L::kPOff + ps * L::kPBytes, &tmap_a, &pfull[ps], (kb >> 1) * 12,
-                        static_cast<int32_t>(row0));
-            ++pit;
-          }
           if (!mbar_wait(&empty[s], ph ^ 1)) {
             ok = false;
             break;
@@ -232,13 +262,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (kA == ASrc::kFp16)
             tma_load_2d(smem + L::kAOff + s * L::kABytes, &tmap_a, &full[s], kb * kTcBK,
                         static_cast<int32_t>(row0));
-          else if (kA == ASrc::kPacked4)
-            tma_load_2d(smem + L::kPOff + s * L::kPBytes, &tmap_a, &full[s], kb * (kTcBK / 8),
-                        static_cast<int32_t>(row0));
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kTcMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = f16_idesc(kTcBM, BN);
@@ -270,10 +297,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_commit(&acc_full[buf]);
       }
     }
-  } else if (warp < 2 + kTcBuilders) {
+  } else if (warp < kTcEpiWarp0 && warp != kTcPackWarp && warp != kTcIdleWarp) {
     // ------------------------------------------------------------------ A builders
     if (kPacked) {
-      const int t = threadIdx.x - 64;          // 0..255
+      // builder index 0..7 of warps 0, 2, 3, 4, 6, 7, 8, 10 (skipping sub-partition 1)
+      const int t = (warp - (warp + 3) / 4) * 32 + lane;   // 0..255
       const int r = t >> 1, h = t & 1;         // tile row, 32-k half of the 64-k stage
       const int64_t N = args.N;
       int64_t it = 0, pit = 0;
@@ -286,24 +314,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int kb = tu.kb0 + i;
           const int s = static_cast<int>(it % S);
           const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-          if ((i & 1) == 0) {    // new group of 128: this row's zero point and scale
+          uint32_t z = 0;
+          __half sv = __float2half(0.0f);
+          if ((i & 1) == 0 && !args.sz_tma) {   // new group of 128, ragged N: from global
             const int64_t g = kb >> 1;
-            const uint32_t z = n < N ? args.zeros[g * N + n] : 0u;
-            const __half sv = n < N ? args.scales[g * N + n] : __float2half(0.0f);
+            if (n < N) {
+              z = args.zeros[g * N + n];
+              sv = args.scales[g * N + n];
+            }
+          }
+          // the A slot is free once the MMA that read it has completed; the X tile of the
+          // stage is not needed here, so building overlaps its load
+          bool got = mbar_wait(&empty[s], ph ^ 1);
+          const int ps = static_cast<int>(pit % P);
+          if (got) got = mbar_wait(&pfull[ps], static_cast<uint32_t>((pit / P) & 1));
+          ok = __all_sync(0xffffffffu, got);   // keep the warp converged for .aligned ops
+          if (!ok) break;
+          const int gi = (i >> 1) % L::kPG;          // group inside the slot
+          if ((i & 1) == 0) {    // this row's zero point and scale for the new group
+            if (args.sz_tma) {   // rows past N were filled with zeros by the TMA unit
+              const uint8_t* sz = smem + L::kSZOff + ps * L::kSZBytes;
+              sv = reinterpret_cast<const __half*>(sz)[gi * kTcBM + r];
+              z = sz[L::kPG * kTcBM * 2 + gi * kTcBM + r];
+            }
             lo = u32_as_h2((0x6400u | z) * 0x00010001u);
             hi = u32_as_h2((0xD400u | (z << 4)) * 0x00010001u);
             sc = __half2half2(sv);
           }
-          bool got = mbar_wait(&full[s], ph) && mbar_wait(&empty[s], ph ^ 1);
-          const int ps = static_cast<int>(pit % kTcPk3Slots);
-          if (kA == ASrc::kPacked3 && got)
-            got = mbar_wait(&pfull[ps], static_cast<uint32_t>((pit / kTcPk3Slots) & 1));
-          ok = __all_sync(0xffffffffu, got);   // keep the warp converged for .aligned ops
-          if (!ok) break;
           uint8_t* atile = smem + L::kAOff + s * L::kABytes;
           if (kA == ASrc::kPacked4) {
-            const uint8_t* ptile = smem + L::kPOff + s * L::kPBytes;
-            const uint4 pw = *reinterpret_cast<const uint4*>(ptile + t * 16);   // row r, half h
+            // row r of group gi: 64 bytes, this stage's 32 k at byte 32 * (i & 1) + 16 * h
+            const uint4 pw = *reinterpret_cast<const uint4*>(
+                smem + L::kPOff + ps * L::kPBytes + r * L::kPRowBytes + gi * 64 + 32 * (i & 1) +
+                16 * h);
             const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -312,7 +355,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
           } else {
             const uint32_t* pw = reinterpret_cast<const uint32_t*>(
-                smem + L::kPOff + ps * L::kPBytes + r * 48 + 12 * (2 * (i & 1) + h));
+                smem + L::kPOff + ps * L::kPBytes + r * L::kPRowBytes + gi * 48 +
+                12 * (2 * (i & 1) + h));
             const uint32_t w0 = pw[0], w1 = pw[1], w2 = pw[2];
             uint4 o;
 #define AWQ_DQ3_CHUNK(I)                                                   \
@@ -326,17 +370,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             AWQ_DQ3_CHUNK(2)
             AWQ_DQ3_CHUNK(3)
 #undef AWQ_DQ3_CHUNK
-            if (i & 1) {                      // both stages of the group are built
-              mbar_arrive(&pempty[ps]);
-              ++pit;
-            }
+          }
+          if (i % (2 * L::kPG) == 2 * L::kPG - 1 || i == tu.nkb - 1) {   // slot consumed
+            mbar_arrive(&pempty[ps]);
+            ++pit;
           }
           fence_proxy_async_smem();
           mbar_arrive(&built[s]);
         }
       }
     }
-  } else {
+  } else if (warp >= kTcEpiWarp0) {
     // ------------------------------------------------------------------ epilogue
     // Warp w reads TMEM lane quarter (w % 4), the only one it may access: 32 weight rows of
     // the finished accumulator, all BN token columns.
@@ -392,11 +436,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);            // the MMA may overwrite this accumulator
     }
+  } else if (kPacked && warp == kTcPackWarp) {
+    // ------------------------------------------------------------------ packed producer
+    if (lane == 0) {
+      int64_t pit = 0;   // group counter, continuous across units
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const TcUnit t = unit_of(u, args);
+        const int32_t row0 = t.row_tile * kTcBM;
+        // a last slot that runs past the unit's K slice loads groups it does not use (zero
+        // filled past K); the transaction count is always the full box
+        for (int i = 0; i < t.nkb; i += 2 * L::kPG, ++pit) {
+          const int g = (t.kb0 + i) >> 1;
+          const int ps = static_cast<int>(pit % P);
+          if (!mbar_wait(&pempty[ps], static_cast<uint32_t>((pit / P) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&pfull[ps], L::kPBytes + (args.sz_tma ? L::kSZBytes : 0));
+          tma_load_2d(smem + L::kPOff + ps * L::kPBytes, &tmap_a, &pfull[ps],
+                      g * (L::kPGroupBytes / 4), row0);
+          if (args.sz_tma) {
+            uint8_t* sz = smem + L::kSZOff + ps * L::kSZBytes;
+            tma_load_2d(sz, &tmap_s, &pfull[ps], row0, g);
+            tma_load_2d(sz + L::kPG * kTcBM * 2, &tmap_z, &pfull[ps], row0, g);
+          }
+        }
+      }
+    }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kTcMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
   }
