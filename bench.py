@@ -471,7 +471,7 @@ def run_b200(args, world, rank, local):
 
     # ---- decode sweep: each (shape, M) on its own
     sweep = []
-    for sh in (shapes if args.only == "all" else []):
+    for sh in (shapes if args.only in ("all", "decode") else []):
         for M in synth.DECODE_M:
             t = time_steps(lambda r, sh=sh, M=M: sh.call(awq, M, r), 200, 10, stream, world)
             b = gemm_bytes(M, sh.N, sh.K)

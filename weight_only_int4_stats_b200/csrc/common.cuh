@@ -68,6 +68,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
   return ok != 0;
 }
 
+// The same test with a suspend-time hint: a thread whose phase is not complete is suspended
+// until the phase completes or about `hint_ns` nanoseconds have passed, instead of spinning
+// and taking issue slots from the warps that are working (a co-resident CTA of the next
+// kernel waits here for the whole of the previous kernel).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar_addr, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kWaitSleepNs = 100000;   // longest single suspension (100 us)
+
 // Waits for the phase with the given parity to complete. Returns false (and flags the
 // status word) if it did not within `limit_ns` (default kWaitLimitNs); the caller then
 // abandons its work.
@@ -77,8 +96,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(a, parity)) return true;
+    if (mbar_try_wait_sleep(a, parity, kWaitSleepNs)) return true;
     if (globaltimer_ns() - t0 > limit_ns) {
       flag_error(kDevErrTimeout);
       return false;

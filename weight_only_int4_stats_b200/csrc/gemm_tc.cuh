@@ -242,16 +242,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == kTcXWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int64_t it = 0;   // stage counter, continuous across units
+      int s = 0;          // stage slot and phase, continuous across units
+      uint32_t ph = 0;
       bool ok = true;
       for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const TcUnit t = unit_of(u, args);
         const int64_t m0 = static_cast<int64_t>(t.m_tile) * BN;
         const int64_t row0 = static_cast<int64_t>(t.row_tile) * kTcBM;
-        for (int i = 0; i < t.nkb; ++i, ++it) {
+        for (int i = 0; i < t.nkb; ++i) {
           const int kb = t.kb0 + i;
-          const int s = static_cast<int>(it % S);
-          const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
           if (!mbar_wait(&empty[s], ph ^ 1)) {
             ok = false;
             break;
@@ -262,6 +261,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (kA == ASrc::kFp16)
             tma_load_2d(smem + L::kAOff + s * L::kABytes, &tmap_a, &full[s], kb * kTcBK,
                         static_cast<int32_t>(row0));
+          if (++s == S) { s = 0; ph ^= 1; }
         }
       }
     }
@@ -269,7 +269,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = f16_idesc(kTcBM, BN);
-      int64_t it = 0, lt = 0;
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t lt = 0;
       bool ok = true;
       for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x, ++lt) {
         const TcUnit t = unit_of(u, args);
@@ -278,9 +280,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!mbar_wait(&acc_empty[buf], acc_ph ^ 1)) break;   // epilogue released the buffer
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-        for (int i = 0; i < t.nkb; ++i, ++it) {
-          const int s = static_cast<int>(it % S);
-          const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+        for (int i = 0; i < t.nkb; ++i) {
           ok = mbar_wait(&full[s], ph);
           if (ok && kPacked) ok = mbar_wait(&built[s], ph);
           if (!ok) break;
@@ -293,6 +293,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                        sw128_kmajor_desc(x_base + kk * 32), idesc, (i | kk) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[s]);
+          if (++s == S) { s = 0; ph ^= 1; }
         }
         tc_commit(&acc_full[buf]);
       }
@@ -304,79 +305,82 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int t = (warp - (warp + 3) / 4) * 32 + lane;   // 0..255
       const int r = t >> 1, h = t & 1;         // tile row, 32-k half of the 64-k stage
       const int64_t N = args.N;
-      int64_t it = 0, pit = 0;
+      int s = 0, ps = 0;      // stage slot and packed slot, with their phases
+      uint32_t ph = 0, pph = 0;
       bool ok = true;
       for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const TcUnit tu = unit_of(u, args);
         const int64_t n = static_cast<int64_t>(tu.row_tile) * kTcBM + r;
-        __half2 lo, hi, sc;
-        for (int i = 0; i < tu.nkb; ++i, ++it) {
+        // one 128-k group per iteration: both of its 64-k stages are built, then one proxy
+        // fence and one arrival per stage (K slices are whole groups, so nkb is even)
+        for (int i = 0; i < tu.nkb; i += 2) {
           const int kb = tu.kb0 + i;
-          const int s = static_cast<int>(it % S);
-          const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
           uint32_t z = 0;
           __half sv = __float2half(0.0f);
-          if ((i & 1) == 0 && !args.sz_tma) {   // new group of 128, ragged N: from global
+          if (!args.sz_tma) {   // ragged N: this row's zero point and scale from global
             const int64_t g = kb >> 1;
             if (n < N) {
               z = args.zeros[g * N + n];
               sv = args.scales[g * N + n];
             }
           }
-          // the A slot is free once the MMA that read it has completed; the X tile of the
-          // stage is not needed here, so building overlaps its load
-          bool got = mbar_wait(&empty[s], ph ^ 1);
-          const int ps = static_cast<int>(pit % P);
-          if (got) got = mbar_wait(&pfull[ps], static_cast<uint32_t>((pit / P) & 1));
+          const int s1 = s + 1 == S ? 0 : s + 1;
+          const uint32_t ph1 = s + 1 == S ? (ph ^ 1u) : ph;
+          // the A slots are free once the MMAs that read them have completed; the X tiles of
+          // the stages are not needed here, so building overlaps their loads
+          bool got = mbar_wait(&empty[s], ph ^ 1) && mbar_wait(&empty[s1], ph1 ^ 1);
+          if (got) got = mbar_wait(&pfull[ps], pph);
           ok = __all_sync(0xffffffffu, got);   // keep the warp converged for .aligned ops
           if (!ok) break;
           const int gi = (i >> 1) % L::kPG;          // group inside the slot
-          if ((i & 1) == 0) {    // this row's zero point and scale for the new group
-            if (args.sz_tma) {   // rows past N were filled with zeros by the TMA unit
-              const uint8_t* sz = smem + L::kSZOff + ps * L::kSZBytes;
-              sv = reinterpret_cast<const __half*>(sz)[gi * kTcBM + r];
-              z = sz[L::kPG * kTcBM * 2 + gi * kTcBM + r];
-            }
-            lo = u32_as_h2((0x6400u | z) * 0x00010001u);
-            hi = u32_as_h2((0xD400u | (z << 4)) * 0x00010001u);
-            sc = __half2half2(sv);
+          if (args.sz_tma) {   // rows past N were filled with zeros by the TMA unit
+            const uint8_t* sz = smem + L::kSZOff + ps * L::kSZBytes;
+            sv = reinterpret_cast<const __half*>(sz)[gi * kTcBM + r];
+            z = sz[L::kPG * kTcBM * 2 + gi * kTcBM + r];
           }
-          uint8_t* atile = smem + L::kAOff + s * L::kABytes;
-          if (kA == ASrc::kPacked4) {
-            // row r of group gi: 64 bytes, this stage's 32 k at byte 32 * (i & 1) + 16 * h
-            const uint4 pw = *reinterpret_cast<const uint4*>(
-                smem + L::kPOff + ps * L::kPBytes + r * L::kPRowBytes + gi * 64 + 32 * (i & 1) +
-                16 * h);
-            const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
+          const __half2 lo = u32_as_h2((0x6400u | z) * 0x00010001u);
+          const __half2 hi = u32_as_h2((0xD400u | (z << 4)) * 0x00010001u);
+          const __half2 sc = __half2half2(sv);
+          const uint8_t* prow = smem + L::kPOff + ps * L::kPBytes + r * L::kPRowBytes;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 o = dequant_word_scaled(words[q], lo, hi, sc);
-              *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + q)) = o;
-            }
-          } else {
-            const uint32_t* pw = reinterpret_cast<const uint32_t*>(
-                smem + L::kPOff + ps * L::kPBytes + r * L::kPRowBytes + gi * 48 +
-                12 * (2 * (i & 1) + h));
-            const uint32_t w0 = pw[0], w1 = pw[1], w2 = pw[2];
-            uint4 o;
+          for (int e = 0; e < 2; ++e) {             // stage i + e of the group
+            uint8_t* atile = smem + L::kAOff + (e ? s1 : s) * L::kABytes;
+            if (kA == ASrc::kPacked4) {
+              // row r of group gi: 64 bytes, this stage's 32 k at byte 32 * e + 16 * h
+              const uint4 pw = *reinterpret_cast<const uint4*>(prow + gi * 64 + 32 * e + 16 * h);
+              const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint4 o = dequant_word_scaled(words[q], lo, hi, sc);
+                *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + q)) = o;
+              }
+            } else {
+              const uint32_t* pw =
+                  reinterpret_cast<const uint32_t*>(prow + gi * 48 + 12 * (2 * e + h));
+              const uint32_t w0 = pw[0], w1 = pw[1], w2 = pw[2];
+              uint4 o;
 #define AWQ_DQ3_CHUNK(I)                                                   \
   o.x = dequant3_pair<I, 0>(w0, w1, w2, lo, sc);                          \
   o.y = dequant3_pair<I, 1>(w0, w1, w2, lo, sc);                          \
   o.z = dequant3_pair<I, 2>(w0, w1, w2, lo, sc);                          \
   o.w = dequant3_pair<I, 3>(w0, w1, w2, lo, sc);                          \
   *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + I)) = o;
-            AWQ_DQ3_CHUNK(0)
-            AWQ_DQ3_CHUNK(1)
-            AWQ_DQ3_CHUNK(2)
-            AWQ_DQ3_CHUNK(3)
+              AWQ_DQ3_CHUNK(0)
+              AWQ_DQ3_CHUNK(1)
+              AWQ_DQ3_CHUNK(2)
+              AWQ_DQ3_CHUNK(3)
 #undef AWQ_DQ3_CHUNK
+            }
           }
-          if (i % (2 * L::kPG) == 2 * L::kPG - 1 || i == tu.nkb - 1) {   // slot consumed
+          if (i % (2 * L::kPG) == 2 * L::kPG - 2 || i == tu.nkb - 2) {   // slot consumed
             mbar_arrive(&pempty[ps]);
-            ++pit;
+            if (++ps == P) { ps = 0; pph ^= 1; }
           }
           fence_proxy_async_smem();
           mbar_arrive(&built[s]);
+          mbar_arrive(&built[s1]);
+          s = s1 + 1 == S ? 0 : s1 + 1;
+          ph = s1 + 1 == S ? (ph1 ^ 1u) : ph1;
         }
       }
     }
@@ -439,17 +443,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (kPacked && warp == kTcPackWarp) {
     // ------------------------------------------------------------------ packed producer
     if (lane == 0) {
-      int64_t pit = 0;   // group counter, continuous across units
+      int ps = 0;        // packed slot and phase, continuous across units
+      uint32_t pph = 0;
       bool ok = true;
       for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const TcUnit t = unit_of(u, args);
         const int32_t row0 = t.row_tile * kTcBM;
         // a last slot that runs past the unit's K slice loads groups it does not use (zero
         // filled past K); the transaction count is always the full box
-        for (int i = 0; i < t.nkb; i += 2 * L::kPG, ++pit) {
+        for (int i = 0; i < t.nkb; i += 2 * L::kPG) {
           const int g = (t.kb0 + i) >> 1;
-          const int ps = static_cast<int>(pit % P);
-          if (!mbar_wait(&pempty[ps], static_cast<uint32_t>((pit / P) & 1) ^ 1)) {
+          if (!mbar_wait(&pempty[ps], pph ^ 1)) {
             ok = false;
             break;
           }
@@ -461,6 +465,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tma_load_2d(sz, &tmap_s, &pfull[ps], row0, g);
             tma_load_2d(sz + L::kPG * kTcBM * 2, &tmap_z, &pfull[ps], row0, g);
           }
+          if (++ps == P) { ps = 0; pph ^= 1; }
         }
       }
     }

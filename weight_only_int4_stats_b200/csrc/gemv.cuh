@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
   if (threadIdx.x == 0) {
     for (int i = 0; i < kG4Slots; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kG4Warps);
+      mbar_init(&empty[i], kG4Warps * 32);
     }
     mbar_init(xfull, 1);
     fence_barrier_init();
@@ -406,33 +406,49 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
   int64_t tile = t0;
   for (int64_t u = 0; u < units; ++u) {
     ok = __all_sync(0xffffffffu, ok && mbar_wait(&full[slot], ph));
+    // Copy this warp's operands of the unit (two groups: packed words of rows r and r + 8,
+    // their scales and zero points) to registers and release the slot at once, so the
+    // producer refills it while this unit is computed: the ring then keeps its full depth
+    // of weight bytes in flight instead of holding a slot through the arithmetic. Every
+    // lane arrives (release semantics), which orders its own shared-memory reads first.
     const uint8_t* sb = slots + slot * kG4SlotBytes;
+    uint4 wA[2], wB[2];
+    uint32_t zAi[2], zBi[2];
+    float scA[2], scB[2];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int gl = 2 * warp + q;               // group inside the unit
+      const uint8_t* wrow = sb + (gl * 16 + 4 * c) * 4;
+      wA[q] = *reinterpret_cast<const uint4*>(wrow + r * (kG4KC / 2));
+      wB[q] = *reinterpret_cast<const uint4*>(wrow + (r + 8) * (kG4KC / 2));
+      const __half* ss = reinterpret_cast<const __half*>(sb + kG4WBytes) + gl * kGemvRows;
+      const uint8_t* zz = sb + kG4WBytes + kG4SBytes + gl * kGemvRows;
+      zAi[q] = zz[r];
+      zBi[q] = zz[r + 8];
+      scA[q] = __half2float(ss[r]);
+      scB[q] = __half2float(ss[r + 8]);
+    }
+    if (ok) mbar_arrive(&empty[slot]);
+    if (++slot == kG4Slots) { slot = 0; ph ^= 1; }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int gl = 2 * warp + q;
       const int g = chunk * kG4Groups + gl;
       if (ok && g < G) {
-        const uint8_t* wrow = sb + (gl * 16 + 4 * c) * 4;
-        const uint4 wA = *reinterpret_cast<const uint4*>(wrow + r * (kG4KC / 2));
-        const uint4 wB = *reinterpret_cast<const uint4*>(wrow + (r + 8) * (kG4KC / 2));
-        const __half* ss = reinterpret_cast<const __half*>(sb + kG4WBytes) + gl * kGemvRows;
-        const uint8_t* zz = sb + kG4WBytes + kG4SBytes + gl * kGemvRows;
-        const uint32_t zAi = zz[r], zBi = zz[r + 8];
-        const float scA = __half2float(ss[r]), scB = __half2float(ss[r + 8]);
         float acc[kNTiles][2][4];
 #pragma unroll
         for (int t = 0; t < kNTiles; ++t)
 #pragma unroll
           for (int i = 0; i < 4; ++i) acc[t][0][i] = acc[t][1][i] = 0.0f;
-        const uint32_t wordsA[4] = {wA.x, wA.y, wA.z, wA.w};
-        const uint32_t wordsB[4] = {wB.x, wB.y, wB.z, wB.w};
+        const uint32_t wordsA[4] = {wA[q].x, wA[q].y, wA[q].z, wA[q].w};
+        const uint32_t wordsB[4] = {wB[q].x, wB[q].y, wB[q].z, wB[q].w};
         const int kx = g * kGroup + 32 * c;
         __half2 loA, hiA, loB, hiB;
         if (!kOffset) {
-          loA = u32_as_h2((0x6400u | zAi) * 0x00010001u);
-          hiA = u32_as_h2((0xD400u | (zAi << 4)) * 0x00010001u);
-          loB = u32_as_h2((0x6400u | zBi) * 0x00010001u);
-          hiB = u32_as_h2((0xD400u | (zBi << 4)) * 0x00010001u);
+          loA = u32_as_h2((0x6400u | zAi[q]) * 0x00010001u);
+          hiA = u32_as_h2((0xD400u | (zAi[q] << 4)) * 0x00010001u);
+          loB = u32_as_h2((0x6400u | zBi[q]) * 0x00010001u);
+          hiB = u32_as_h2((0xD400u | (zBi[q] << 4)) * 0x00010001u);
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -461,23 +477,20 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
 #pragma unroll
           for (int i = 0; i < 4; ++i) d[i] = acc[t][0][i] + acc[t][1][i];
           if (kOffset) {
-            const float zA = static_cast<float>(zAi), zB = static_cast<float>(zBi);
+            const float zA = static_cast<float>(zAi[q]), zB = static_cast<float>(zBi[q]);
             const float4 cm = *reinterpret_cast<const float4*>(cc + (g * kTok + 8 * t + 2 * c) * 2);
             d[0] -= fmaf(zA, cm.y, cm.x);
             d[1] -= fmaf(zA, cm.w, cm.z);
             d[2] -= fmaf(zB, cm.y, cm.x);
             d[3] -= fmaf(zB, cm.w, cm.z);
           }
-          total[t][0] = fmaf(scA, d[0], total[t][0]);
-          total[t][1] = fmaf(scA, d[1], total[t][1]);
-          total[t][2] = fmaf(scB, d[2], total[t][2]);
-          total[t][3] = fmaf(scB, d[3], total[t][3]);
+          total[t][0] = fmaf(scA[q], d[0], total[t][0]);
+          total[t][1] = fmaf(scA[q], d[1], total[t][1]);
+          total[t][2] = fmaf(scB[q], d[2], total[t][2]);
+          total[t][3] = fmaf(scB[q], d[3], total[t][3]);
         }
       }
     }
-    __syncwarp();
-    if (ok && lane == 0) mbar_arrive(&empty[slot]);
-    if (++slot == kG4Slots) { slot = 0; ph ^= 1; }
 
     if (chunk == C - 1) {
       // tile complete: fixed-order sum over the eight consumer warps, fp16 store
