@@ -361,6 +361,39 @@ def test_decode_chain_output_feeds_next_input(awq):
     assert rel_fro(Y2.float().cpu().numpy(), o2) <= GEMM_RTOL
 
 
+@pytest.mark.parametrize("M,N,K", [(64, 1024, 1024), (64, 1000, 1024), (40, 512, 2304),
+                                   (300, 768, 512)])
+def test_tensor_core_gemm_right_after_quantize_on_same_stream(awq, M, N, K):
+    # The tensor-core GEMM may also start before the previous kernel on the stream ends; its
+    # packed weights, scales and zero points (read by TMA, or by the builders when N % 16 != 0)
+    # and the split-K partials must all come from after that kernel.
+    W, X, m = rand_layer(707 + N, N, K, M)
+    s = np.sqrt(m).astype(np.float32)
+    Wd, sd, Xd = cu(W), cu(s), cu(X)
+    for _ in range(3):
+        qw, sc, z = awq.awq_quantize_pack(Wd, sd, 4)
+        Y = awq.awq_gemm_w4a16(Xd, qw, sc, z, N, K)
+    oq, osc, oz = O.quantize_pack(W, s, 4, 128)
+    want = O.gemm_w4a16(X, oq, osc, oz, N, K, 4, 128)
+    assert rel_fro(Y.float().cpu().numpy(), want) <= GEMM_RTOL
+
+
+def test_tensor_core_chain_output_feeds_next_input(awq):
+    # Y1 = X W1^T, Y2 = Y1 W2^T back to back on the tensor-core path.
+    M, K1, N1, N2 = 96, 1024, 1536, 512
+    W1, X, m = rand_layer(808, N1, K1, M)
+    W2, _, _ = rand_layer(809, N2, N1, M)
+    p1 = O.quantize_pack(W1, None, 4, 128)
+    p2 = O.quantize_pack(W2, None, 4, 128)
+    d1 = [cu(a) for a in p1]
+    d2 = [cu(a) for a in p2]
+    Y1 = awq.awq_gemm_w4a16(cu(X), *d1, N1, K1)
+    Y2 = awq.awq_gemm_w4a16(Y1, *d2, N2, N1)
+    o1 = O.gemm_w4a16(X, *p1, N1, K1, 4, 128).astype(np.float16)
+    o2 = O.gemm_w4a16(o1, *p2, N2, N1, 4, 128)
+    assert rel_fro(Y2.float().cpu().numpy(), o2) <= GEMM_RTOL
+
+
 # ----------------------------------------------------------------------------- failure detection
 
 def test_bounded_wait_times_out_and_reports(awq):

@@ -132,7 +132,17 @@ awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_ro
   const int64_t units = static_cast<int64_t>(a.m_tiles) * a.row_tiles * a.k_splits;
   const int64_t sms = num_sms();
   const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);   // persistent
-  kern<<<grid, awq::kTcThreads, L::kSmem, st>>>(tx, ta, ts, tz, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(awq::kTcThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(L::kSmem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tx, ta, ts, tz, a) != cudaSuccess) return AWQ_ERR_CUDA;
   return launch_status();
 }
 

@@ -238,6 +238,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Programmatic dependent launch: the setup above may overlap the previous kernel on the
+  // stream; every thread waits for that kernel's completion (and memory) before its first
+  // global access, and lets the next kernel launch early.
+  pdl_launch_dependents();
+  pdl_wait();
 
   if (warp == kTcXWarp) {
     // ------------------------------------------------------------------ TMA producer
