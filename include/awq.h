@@ -157,10 +157,12 @@ AWQ_API awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, cons
  *     Y[m, n] = sum_k x'[m, k] * (q[n, k] - z[k/128, n]) * scale[k/128, n]
  * with x' = X, or x' = fp16(X[m, k] * inv_s[k]) when inv_s is not NULL (the activation side
  * of the per-channel scaling). fp32 accumulation, fp16 output.
- * M <= 16 with 4 bits runs the decode kernel (HBM-bound GEMV); larger M (and 3 bits) the
- * tensor-core kernel. X: fp16 [M, K]; Y: fp16 [M, N]. M = 0 or N = 0 is a no-op.
- * workspace: at least awq_gemm_workspace_size(M, N, K, bits) bytes (0 when inv_s is NULL
- * or M <= 16). */
+ * M <= 16 with 4 bits runs a decode kernel (HBM-bound GEMV; for 8 < M <= 16 only when X
+ * fits in one CTA's shared memory); other calls (and 3 bits) run the tensor-core kernel.
+ * X: fp16 [M, K]; Y: fp16 [M, N]. M = 0 or N = 0 is a no-op.
+ * workspace: at least awq_gemm_workspace_size(M, N, K, bits) bytes: 0 for the decode
+ * kernels, otherwise room for x' and, when K is split across CTAs, the fp32 partial sums
+ * (the size does not depend on whether inv_s is given). */
 AWQ_API size_t awq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits);
 AWQ_API awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
                           const awq_f16* scales, const uint8_t* zeros, int64_t N, int64_t K,

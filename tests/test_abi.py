@@ -93,3 +93,15 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(awq, "_lib", None)
     with pytest.raises(ImportError):
         awq.lib()
+
+
+def test_gemm_workspace_follows_the_chosen_kernel():
+    # the decode kernels need no workspace; an 8 < M <= 16 call whose X does not fit the
+    # streaming kernel's shared memory takes the tensor-core path and needs room for x'
+    L = _lib()
+    assert L.awq_gemm_workspace_size(1, 4096, 11008, 4) == 0
+    assert L.awq_gemm_workspace_size(8, 4096, 11008, 4) == 0
+    assert L.awq_gemm_workspace_size(16, 4096, 4096, 4) == 0
+    assert L.awq_gemm_workspace_size(16, 4096, 11008, 4) >= 16 * 11008 * 2
+    assert L.awq_gemm_workspace_size(16, 4104, 4096, 4) >= 16 * 4096 * 2   # N % 16 != 0
+    assert L.awq_gemm_workspace_size(64, 4096, 4096, 4) >= 64 * 4096 * 2

@@ -160,14 +160,22 @@ awq_status launch_tc_bn(const __half* Xop, int64_t M, const void* Aop, int64_t a
 // memory, or N is not a multiple of 16); the caller then uses the register-streaming kernel.
 constexpr int kSmemLimit = 232448;   // 227 KB per CTA on sm_100
 
+// Whether the streaming decode kernel takes this shape: N in whole 16-row tiles and X plus
+// the weight ring within one CTA's shared memory (kNTiles = 1 for M <= 8, 2 for M <= 16).
+bool gemv_stream_fits(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || M > 16 || N % 16 != 0 || K / awq::kGroup > 65535) return false;
+  if (M * K * 2 > kSmemLimit) return false;
+  const int nt = M <= 8 ? 1 : 2;
+  return awq::G4Smem::make(static_cast<int>(M), K, nt).total(nt) <= kSmemLimit;
+}
+
 template <int kNTiles, bool kOffset>
 awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweight,
                               const __half* scales, const uint8_t* zeros, int64_t N, int64_t K,
                               const float* inv_s, __half* y, cudaStream_t st) {
-  if (N % 16 != 0 || K / awq::kGroup > 65535) return AWQ_ERR_UNSUPPORTED;
+  if (!gemv_stream_fits(M, N, K)) return AWQ_ERR_UNSUPPORTED;
   const awq::G4Smem lay = awq::G4Smem::make(static_cast<int>(M), K, kNTiles);
   const int smem = lay.total(kNTiles);
-  if (smem > kSmemLimit) return AWQ_ERR_UNSUPPORTED;
   static bool attr_set[kMaxDevices] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
@@ -494,7 +502,9 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
 // ------------------------------------------------------------------ GEMM
 size_t awq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits) {
   if (M <= 0 || K <= 0 || N <= 0) return 0;
-  if (M <= 16 && bits == 4) return 0;
+  // the decode kernels need none; 8 < M <= 16 with an X too large for the streaming kernel
+  // takes the tensor-core path below
+  if (M <= 16 && bits == 4 && (M <= 8 || gemv_stream_fits(M, N, K))) return 0;
   const int splits = splitk_for(M, N, K);
   size_t bytes = align256(static_cast<size_t>(M) * K * sizeof(__half));   // x * inv_s
   if (splits > 1) bytes += align256(static_cast<size_t>(splits) * M * N * sizeof(float));
@@ -524,14 +534,14 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
         : M <= 8 ? launch_gemv_stream<1, false>(x, M, qweight, sc, zeros, N, K, inv_s, y, st)
                  : launch_gemv_stream<2, false>(x, M, qweight, sc, zeros, N, K, inv_s, y, st);
     if (r != AWQ_ERR_UNSUPPORTED) return r;
-    const unsigned grid = static_cast<unsigned>((N + awq::kGemvRows - 1) / awq::kGemvRows);
-    if (M <= 8)
+    // the streaming kernel cannot hold X (or N % 16 != 0): register streaming for M <= 8,
+    // the tensor-core path below for 8 < M <= 16
+    if (M <= 8) {
+      const unsigned grid = static_cast<unsigned>((N + awq::kGemvRows - 1) / awq::kGemvRows);
       awq::gemv_w4a16_kernel<1><<<grid, awq::kGemvWarps * 32, 0, st>>>(
           x, static_cast<int>(M), qweight, sc, zeros, N, K, inv_s, y);
-    else
-      awq::gemv_w4a16_kernel<2><<<grid, awq::kGemvWarps * 32, 0, st>>>(
-          x, static_cast<int>(M), qweight, sc, zeros, N, K, inv_s, y);
-    return launch_status();
+      return launch_status();
+    }
   }
   if ((N + awq::kTcBM - 1) / awq::kTcBM > 65535) return AWQ_ERR_INVALID_ARG;
   const __half* xop = x;

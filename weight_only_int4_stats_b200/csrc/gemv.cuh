@@ -336,46 +336,38 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
   // runs every named barrier, so the consumer warps cannot deadlock one another.
   const int r = lane >> 2, c = lane & 3;
   bool ok = __all_sync(0xffffffffu, mbar_wait(xfull, 0));
-  if (inv_s != nullptr || kOffset) {
-    // x <- fp16(x * inv_s); for kOffset also divide columns k%8 in {2,3,6,7} by 16
-    const int n8 = M * Ki / 8;
-    for (int i = threadIdx.x; ok && i < n8; i += kG4Warps * 32) {
-      uint4 v = reinterpret_cast<uint4*>(xs)[i];
-      if (inv_s != nullptr) {
-        const int k = (i * 8) % Ki;
-        const float4 s0 = *reinterpret_cast<const float4*>(inv_s + k);
-        const float4 s1 = *reinterpret_cast<const float4*>(inv_s + k + 4);
-        float2 f;
-        f = __half22float2(u32_as_h2(v.x)); v.x = h2_as_u32(__floats2half2_rn(f.x * s0.x, f.y * s0.y));
-        f = __half22float2(u32_as_h2(v.y)); v.y = h2_as_u32(__floats2half2_rn(f.x * s0.z, f.y * s0.w));
-        f = __half22float2(u32_as_h2(v.z)); v.z = h2_as_u32(__floats2half2_rn(f.x * s1.x, f.y * s1.y));
-        f = __half22float2(u32_as_h2(v.w)); v.w = h2_as_u32(__floats2half2_rn(f.x * s1.z, f.y * s1.w));
-      }
-      if (kOffset) {
-        const __half2 sixteenth = __float2half2_rn(0.0625f);
-        v.y = h2_as_u32(__hmul2(u32_as_h2(v.y), sixteenth));
-        v.w = h2_as_u32(__hmul2(u32_as_h2(v.w), sixteenth));
-      }
-      reinterpret_cast<uint4*>(xs)[i] = v;
-    }
-    named_bar_sync(1, kG4Warps * 32);
-  }
   if (kOffset) {
-    // C1 = 1024 * sum(xs), C2 = sum(x) per (group, token < M); tokens >= M get zeros.
-    // 8 threads per (group, token) pair, 4 pairs per warp and pass, three xor-shuffles.
+    // One pass over X: x <- fp16(x * inv_s), columns k%8 in {2,3,6,7} divided by 16 (exact
+    // in fp16), and per (group, token < M) C1 = 1024 * sum(xs) and C2 = sum(x) from the staged
+    // values; tokens >= M get zeros. 8 threads per (group, token) pair, 2 chunks of 8 each,
+    // 4 pairs per warp and pass, three xor-shuffles.
     const int sub = lane & 7;
     const int npairs = G * M;
+    const __half2 sixteenth = __float2half2_rn(0.0625f);
     for (int base = warp * 4; base < npairs; base += kG4Warps * 4) {
       const int pr = base + (lane >> 3);
       const bool live = ok && pr < npairs;
       const int g = live ? pr / M : 0, m = live ? pr % M : 0;
-      const uint4* src = reinterpret_cast<const uint4*>(xs + m * Ki + g * kGroup + 16 * sub);
+      uint4* src = reinterpret_cast<uint4*>(xs + m * Ki + g * kGroup + 16 * sub);
       float c1 = 0.0f, c2 = 0.0f;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const uint4 u = src[h];
-        const float2 lx = __half22float2(u32_as_h2(u.x)), hy = __half22float2(u32_as_h2(u.y));
-        const float2 lz = __half22float2(u32_as_h2(u.z)), hw = __half22float2(u32_as_h2(u.w));
+        uint4 v = live ? src[h] : make_uint4(0u, 0u, 0u, 0u);
+        if (inv_s != nullptr && live) {
+          const int k = g * kGroup + 16 * sub + 8 * h;
+          const float4 s0 = *reinterpret_cast<const float4*>(inv_s + k);
+          const float4 s1 = *reinterpret_cast<const float4*>(inv_s + k + 4);
+          float2 f;
+          f = __half22float2(u32_as_h2(v.x)); v.x = h2_as_u32(__floats2half2_rn(f.x * s0.x, f.y * s0.y));
+          f = __half22float2(u32_as_h2(v.y)); v.y = h2_as_u32(__floats2half2_rn(f.x * s0.z, f.y * s0.w));
+          f = __half22float2(u32_as_h2(v.z)); v.z = h2_as_u32(__floats2half2_rn(f.x * s1.x, f.y * s1.y));
+          f = __half22float2(u32_as_h2(v.w)); v.w = h2_as_u32(__floats2half2_rn(f.x * s1.z, f.y * s1.w));
+        }
+        v.y = h2_as_u32(__hmul2(u32_as_h2(v.y), sixteenth));
+        v.w = h2_as_u32(__hmul2(u32_as_h2(v.w), sixteenth));
+        if (live) src[h] = v;
+        const float2 lx = __half22float2(u32_as_h2(v.x)), hy = __half22float2(u32_as_h2(v.y));
+        const float2 lz = __half22float2(u32_as_h2(v.z)), hw = __half22float2(u32_as_h2(v.w));
         const float lo = (lx.x + lx.y) + (lz.x + lz.y), hi = (hy.x + hy.y) + (hw.x + hw.y);
         c1 += lo + hi;
         c2 += lo + 16.0f * hi;
@@ -392,6 +384,22 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
     }
     for (int i = threadIdx.x; i < G * kTok; i += kG4Warps * 32)
       if (i % kTok >= M) { cc[2 * i] = 0.0f; cc[2 * i + 1] = 0.0f; }
+    named_bar_sync(1, kG4Warps * 32);
+  } else if (inv_s != nullptr) {
+    // x <- fp16(x * inv_s)
+    const int n8 = M * Ki / 8;
+    for (int i = threadIdx.x; ok && i < n8; i += kG4Warps * 32) {
+      uint4 v = reinterpret_cast<uint4*>(xs)[i];
+      const int k = (i * 8) % Ki;
+      const float4 s0 = *reinterpret_cast<const float4*>(inv_s + k);
+      const float4 s1 = *reinterpret_cast<const float4*>(inv_s + k + 4);
+      float2 f;
+      f = __half22float2(u32_as_h2(v.x)); v.x = h2_as_u32(__floats2half2_rn(f.x * s0.x, f.y * s0.y));
+      f = __half22float2(u32_as_h2(v.y)); v.y = h2_as_u32(__floats2half2_rn(f.x * s0.z, f.y * s0.w));
+      f = __half22float2(u32_as_h2(v.z)); v.z = h2_as_u32(__floats2half2_rn(f.x * s1.x, f.y * s1.y));
+      f = __half22float2(u32_as_h2(v.w)); v.w = h2_as_u32(__floats2half2_rn(f.x * s1.z, f.y * s1.w));
+      reinterpret_cast<uint4*>(xs)[i] = v;
+    }
     named_bar_sync(1, kG4Warps * 32);
   }
 
