@@ -56,7 +56,7 @@ def peaks():
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
 # the current kernels on these workloads: the three M = 1 decode launches of a step, averaged,
 # and the 4-bit M = 2048 [28672, 8192] prefill launch. Set to None when a kernel changes.
-DECODE_TRAFFIC_PER_LAUNCH = None   # decode kernel changed since its last capture
+DECODE_TRAFFIC_PER_LAUNCH = (8.812288e6 + 23.631616e6 + 23.645440e6) / 3
 PREFILL_TRAFFIC_PER_LAUNCH = 0.209463296e9 + 0.101155072e9
 
 
