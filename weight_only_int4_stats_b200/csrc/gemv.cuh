@@ -1,4 +1,7 @@
 // K3: W4A16 decode GEMM for M <= 16 tokens, Y[m, n] = sum_k x[m, k] * deq[n, k].
+// Two kernels: the register-streaming kernel below, which takes M <= 8 calls that the
+// streaming kernel further down cannot (N % 16 != 0, or X larger than its shared memory),
+// and the TMA-fed streaming kernel, the default.
 //
 // builderai.tools "AWQ", "About" (kernels for 4-bit weights with 16-bit activations) and
 // robotsatlas.com "AWQ", "Implementation pitfalls: Missing matched inference kernels"
@@ -193,7 +196,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_w4a16_kernel(
 namespace awq {
 
 // ---------------------------------------------------------------------------------------
-// Streaming decode GEMM (the default decode path for M <= 16 when X fits in shared memory).
+// Streaming decode GEMM (the decode path for M <= 16 when X fits in shared memory; an
+// 8 < M <= 16 call whose X does not fit takes the tensor-core GEMM instead).
 //
 // Persistent: the grid is sized to the resident capacity and CTA b owns the contiguous
 // range of whole 16-row tiles [b*T/P, (b+1)*T/P), so no output is split across CTAs and the
@@ -209,14 +213,17 @@ namespace awq {
 //
 // Eight consumer warps each take two 128-wide groups of every unit (two independent MMA
 // chains) with register-only dequantization feeding mma.sync m16n8k16 (weights as the
-// 16-row A operand, activations as the 8-column B operand). Two dequantization forms:
+// 16-row A operand, activations as the 8-column B operand). A warp copies its packed
+// words, scales and zero points of the unit to registers and releases the ring slot
+// before the arithmetic, so the producer can refill it at once. Two dequantization forms:
 //  * M = 1 (kOffset): a mask-and-or with 0x6400 turns the nibble pair (k0, k1) of a word
 //    into the exact fp16 values (1024 + q0, 1024 + q1) and the pair (k2, k3), stored 4 bits
 //    higher, into (1024 + 16 q2, 1024 + 16 q3) (the same after a shift by 8 for k4..k7);
 //    these go to the MMA unchanged against X staged with columns k%8 in {2,3,6,7} divided by
 //    16 (exact in fp16), so per group the MMA returns sum_k x_k q_k + C1 with
 //    C1 = 1024 * sum_k xs_k; with C2 = sum_k x_k the group adds s * (mma - C1 - z C2).
-//    C1 and C2 are computed once per CTA. Five integer operations per packed word; the fp32
+//    The staging and C1, C2 are one pass over X per CTA. Five integer operations per
+//    packed word; the fp32
 //    cancellation of the 1024 offset keeps about 13 significant bits of each group sum.
 //  * M > 1: one fp16 subtract (or multiply-add) per pair leaves the exact q - z first.
 // Per-tile sums of the eight warps are added in a fixed order and stored as fp16.
