@@ -512,7 +512,7 @@ def run_b200(args, world, rank, local):
     # ---- batched decode / small prefill: M in 32..256 on the batched shapes (weights > L2 in
     #      rotation), GB/s and TFLOP/s per (shape, M)
     batched = []
-    for (N, K) in (synth.BATCHED_SHAPES if args.only == "all" else []):
+    for (N, K) in (synth.BATCHED_SHAPES if args.only in ("all", "batched") else []):
         W, mag, X = synth.batched_layer(N, K)
         s_ = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(dev)
         Wt = torch.from_numpy(W).to(dev)
@@ -538,7 +538,7 @@ def run_b200(args, world, rank, local):
     # ---- prefill at M = 2048 (4-bit on the three shapes, then the 3-bit variant)
     prefill = []
     pf_cases = [(N, K, 4) for (N, K) in synth.PREFILL_SHAPES] + [(*synth.PREFILL_SHAPES[0], 3)]
-    for (N, K, bits) in (pf_cases if args.only != "decode" else []):
+    for (N, K, bits) in (pf_cases if args.only not in ("decode", "batched") else []):
         W, mag, X = synth.prefill_layer(N, K, 2048)
         s = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(dev)
         Wd = torch.from_numpy(W).to(dev)
@@ -614,7 +614,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--only", choices=["all", "decode", "prefill", "rows", "profile"],
+    ap.add_argument("--only", choices=["all", "decode", "batched", "prefill", "rows", "profile"],
                     default="all",
                     help="run one section only (used by the profiling commands)")
     args = ap.parse_args()
