@@ -67,14 +67,19 @@ def gemm_bytes(M, N, K, bits=4):
 # ----------------------------------------------------------------------------- distributed
 
 def dist_setup():
+    """One process per GPU under torchrun (RANK / LOCAL_RANK / WORLD_SIZE / MASTER_*): NCCL
+    on GPUs; gloo on a host without one (the replica bookkeeping is the same)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -90,9 +95,17 @@ def max_over_ranks(x, world):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_rate(units_per_rank, seconds, world):
+    """Whole-job rate: the units all ranks processed over the slowest rank's time (every
+    rank runs the same fixed work). Returns (rate, slowest time)."""
+    t_max = max_over_ranks(seconds, world)
+    return units_per_rank * world / t_max, t_max
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -464,8 +477,7 @@ def run_b200(args, world, rank, local):
     clocks.start()
     dt = time_steps(step, args.steps, args.warmup, stream, world)
     clk = clocks.stop()
-    dt_max = max_over_ranks(dt, world)
-    value = step_bytes * args.steps * world / dt_max / 1e9
+    value, dt_max = job_rate(step_bytes * args.steps / 1e9, dt, world)
     per_gpu = step_bytes * args.steps / dt / 1e9
     launches = args.steps * len(shapes)
 
