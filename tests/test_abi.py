@@ -105,3 +105,17 @@ def test_gemm_workspace_follows_the_chosen_kernel():
     assert L.awq_gemm_workspace_size(16, 4096, 11008, 4) >= 16 * 11008 * 2
     assert L.awq_gemm_workspace_size(16, 4104, 4096, 4) >= 16 * 4096 * 2   # N % 16 != 0
     assert L.awq_gemm_workspace_size(64, 4096, 4096, 4) >= 64 * 4096 * 2
+
+
+def test_gemm_workspace_is_checked_before_launch():
+    # the tensor-core path with inv_s needs room for x'; a missing or short workspace is
+    # rejected on the host (AWQ_ERR_WORKSPACE) before anything is launched
+    L = _lib()
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    need = L.awq_gemm_workspace_size(64, 4096, 4096, 4)
+    assert need >= 64 * 4096 * 2
+    assert L.awq_gemm_w4a16(fake, 64, fake, fake, fake, 4096, 4096, 4, 128, fake, fake, None,
+                            0, None) == 3
+    assert L.awq_gemm_w4a16(fake, 64, fake, fake, fake, 4096, 4096, 4, 128, fake, fake, fake,
+                            64 * 4096 * 2 - 16, None) == 3
