@@ -99,12 +99,13 @@ AWQ_API awq_status awq_act_stats(const awq_f16* X, int64_t M, int64_t K, float* 
  * provide a workspace: a plugin inside another framework's engine that is handed only its
  * input and output pointers, or a latency-critical path that must not call cudaMalloc
  * (which can synchronize the whole device).
- * Instead of a workspace it uses one 4 MiB array of device memory that the library defines
+ * Instead of a workspace it uses one 1 MiB array of device memory that the library defines
  * at file scope; every GPU that loads the library holds that array until the process exits.
  * Limits: K <= 65536 (K a multiple of 8, M >= 1); a larger K returns AWQ_ERR_INVALID_ARG
- * before anything is launched. The row split is capped so the partial sums fit the array,
- * which can change the fp64 summation order relative to awq_act_stats (the results agree
- * whenever those sums are exact, as they are for fp16 inputs of moderate range).
+ * before anything is launched. The row split is capped at 2^17 / K slices so the partial
+ * sums fit the array (on a 148-SM B200 the cap binds for K = 4096 once M > 2048), which can
+ * change the fp64 summation order relative to awq_act_stats (the results agree whenever
+ * those sums are exact, as they are for fp16 inputs of moderate range).
  * The first call on each device looks up the array's device address (with that device
  * current) and caches it; make that first call before any stream capture.
  * Every call shares the one array: calls that may overlap on the GPU (different streams,

@@ -45,19 +45,40 @@ def _noalloc_version(L, X, K, stream):
     return out
 
 
-@pytest.mark.parametrize("M,K", [(256, 512), (4097, 4096), (65536, 4096)])
+def _activations(M, K, seed):
+    rng = np.random.default_rng(seed)
+    mag = rng.lognormal(0.0, 0.7, K).astype(np.float32)
+    return torch.from_numpy((rng.standard_normal((M, K), dtype=np.float32) * mag)
+                            .astype(np.float16)).cuda()
+
+
+# On a 148-SM B200 the array (2^17 doubles) caps the row split at 2^17 / K slices: the
+# 4097 x 4096 and 65536 x 4096 calls want 65 and 74 slices and get 32, the 2048 x 65536
+# call wants 5 and gets 2; the 256 x 512 call (4 slices) is below its cap of 256.
+@pytest.mark.parametrize("M,K", [(256, 512), (4097, 4096), (65536, 4096), (2048, 65536)])
 def test_noalloc_matches_workspace_entry_point_twice(lib, M, K):
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    rng = np.random.default_rng(M + K)
-    mag = rng.lognormal(0.0, 0.7, K).astype(np.float32)
-    X = torch.from_numpy((rng.standard_normal((M, K), dtype=np.float32) * mag)
-                         .astype(np.float16)).cuda()
+    X = _activations(M, K, M + K)
     want = _workspace_version(lib, X, K, stream).cpu().numpy()
     # two calls in a row: the second runs on the array the first one left behind
     first = _noalloc_version(lib, X, K, stream).cpu().numpy()
     second = _noalloc_version(lib, X, K, stream).cpu().numpy()
     np.testing.assert_array_equal(first, want)
     np.testing.assert_array_equal(second, want)
+
+
+def test_noalloc_small_call_after_large_call_on_other_data(lib):
+    # A large call fills most of the array with its partial sums; a smaller call on different
+    # data (fewer slices, smaller K) must not pick any of them up.
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    big = _activations(65536, 4096, 11)
+    small = _activations(300, 1024, 12)
+    want_big = _workspace_version(lib, big, 4096, stream).cpu().numpy()
+    want_small = _workspace_version(lib, small, 1024, stream).cpu().numpy()
+    got_big = _noalloc_version(lib, big, 4096, stream).cpu().numpy()
+    got_small = _noalloc_version(lib, small, 1024, stream).cpu().numpy()
+    np.testing.assert_array_equal(got_big, want_big)
+    np.testing.assert_array_equal(got_small, want_small)
 
 
 def test_noalloc_rejects_k_beyond_its_array(lib):

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "awq.h"
@@ -31,17 +32,19 @@ awq_status launch_status() {
   return e == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
+// Per-device caches below are atomics: host threads may call the library concurrently, and
+// a value computed twice is the same value, so a racing first call only repeats work.
 int num_sms() {
-  static int cache[kMaxDevices] = {0};
+  static std::atomic<int> cache[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  if (cache[dev] == 0) {
-    int v = 0;
+  int v = cache[dev].load(std::memory_order_acquire);
+  if (v == 0) {
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
       v = 148;
-    cache[dev] = v;
+    cache[dev].store(v, std::memory_order_release);
   }
-  return cache[dev];
+  return v;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda).
@@ -84,15 +87,15 @@ template <int BN, ASrc kA, Epi kEpi>
 awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_rows,
                      const awq::TcArgs& args, cudaStream_t st) {
   using L = awq::TcLayout<BN, kA>;
-  static bool attr_set[kMaxDevices] = {false};
+  static std::atomic<bool> attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
   auto kern = awq::tc_gemm_kernel<BN, kA, kEpi>;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem) !=
         cudaSuccess)
       return AWQ_ERR_CUDA;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   CUtensorMap tx, ta;
   if (!make_tmap_2d(&tx, Xop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, args.K, BN, awq::kTcBK,
@@ -176,15 +179,15 @@ awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweigh
   if (!gemv_stream_fits(M, N, K)) return AWQ_ERR_UNSUPPORTED;
   const awq::G4Smem lay = awq::G4Smem::make(static_cast<int>(M), K, kNTiles);
   const int smem = lay.total(kNTiles);
-  static bool attr_set[kMaxDevices] = {false};
+  static std::atomic<bool> attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
   auto kern = awq::gemv_stream_kernel<kNTiles, kOffset>;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
         cudaSuccess)
       return AWQ_ERR_CUDA;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, awq::kG4Threads, smem) !=
@@ -319,8 +322,8 @@ awq_status awq_act_stats(const awq_f16* X, int64_t M, int64_t K, float* s_x, voi
 // process exits. In host code the name is only a stand-in for the symbol, so its device
 // address is looked up once per device (with that device current) and cached.
 namespace {
-constexpr int64_t kNoAllocScratchDoubles = int64_t{1} << 19;   // 4 MiB
-constexpr int64_t kNoAllocMaxK = 65536;                       // >= 8 row slices per call
+constexpr int64_t kNoAllocScratchDoubles = int64_t{1} << 17;   // 1 MiB
+constexpr int64_t kNoAllocMaxK = 65536;                       // >= 2 row slices per call
 static __device__ __align__(256) double g_noalloc_scratch[kNoAllocScratchDoubles];
 
 double* g_noalloc_ptr[kMaxDevices] = {nullptr};

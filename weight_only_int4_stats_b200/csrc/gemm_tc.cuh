@@ -497,8 +497,9 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int k_sp
     }
     *reinterpret_cast<__half2*>(Y + i) = __floats2half2_rn(acc.x, acc.y);
     *reinterpret_cast<__half2*>(Y + i + 2) = __floats2half2_rn(acc.z, acc.w);
-  } else {
-    for (int64_t e = i; e < MN; ++e) {
+  } else {   // this thread's four outputs, one at a time
+    const int64_t end = i + 4 < MN ? i + 4 : MN;
+    for (int64_t e = i; e < end; ++e) {
       float acc = partial[e];
       for (int s = 1; s < k_splits; ++s) acc += partial[static_cast<int64_t>(s) * MN + e];
       Y[e] = __float2half_rn(acc);
