@@ -53,11 +53,40 @@ def peaks():
             "source": "fallback"}
 
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of
-# the current kernels on these workloads: the three M = 1 decode launches of a step, averaged,
-# and the 4-bit M = 2048 [28672, 8192] prefill launch. Set to None when a kernel changes.
-DECODE_TRAFFIC_PER_LAUNCH = (8.812288e6 + 23.631616e6 + 23.645440e6) / 3
-PREFILL_TRAFFIC_PER_LAUNCH = 0.209463296e9 + 0.101155072e9
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) come from the committed
+# ncu summaries under profiles/: a summary states them on a line
+#   bench-traffic: <kernel> <bytes per launch> <sha256 prefix of the kernel's source files>
+# and the figure is used only while the sources still hash to that value (else null: the
+# kernel changed since the counters were taken).
+KERNEL_SOURCES = {
+    "gemv_stream_decode_M1": ["gemv.cuh", "common.cuh"],
+    "tc_gemm_prefill_28672x8192_M2048": ["gemm_tc.cuh", "common.cuh"],
+}
+
+
+def source_hash(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "weight_only_int4_stats_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel):
+    """(bytes per launch, note) from the profile summaries, or (None, why not)."""
+    want = source_hash(kernel)
+    pdir = os.path.join(ROOT, "profiles")
+    seen = False
+    for name in sorted(os.listdir(pdir)) if os.path.isdir(pdir) else []:
+        with open(os.path.join(pdir, name)) as f:
+            for line in f:
+                parts = line.strip().strip("`").split()
+                if len(parts) == 4 and parts[0] == "bench-traffic:" and parts[1] == kernel:
+                    seen = True
+                    if parts[3] == want:
+                        return float(parts[2]), f"profiles/{name}"
+    return None, ("kernel changed since its ncu capture" if seen else "no ncu capture")
 
 
 def gemm_bytes(M, N, K, bits=4):
@@ -179,9 +208,11 @@ class DecodeShape:
         self.Yh = torch.empty(m_max, N, dtype=torch.float16).pin_memory()
 
     def call(self, awq, M, r, stream=None):
+        # the packed weights are static (no kernel writes them between steps), which is the
+        # AWQ_GEMM_WEIGHTS_READY contract: each GEMM may stream them while the previous runs
         qw, sc, z = self.w[r % self.copies]
         awq.awq_gemm_w4a16(self.X[:M], qw, sc, z, self.N, self.K, 4, out=self.Y[:M],
-                           stream=stream)
+                           stream=stream, weights_ready=True)
 
 
 def capture_run(fn_per_step, first, count, stream):
@@ -217,31 +248,39 @@ def time_steps(fn_per_step, steps, warmup, stream, world):
     return e0.elapsed_time(e1) / 1e3   # seconds
 
 
-def cpu_oracle_sample(shapes, rows=512, repeats=2):
-    """The oracle (numpy, fp64) on a row slice of each decode shape at M = 1, one BLAS
-    thread. Returns (GB/s of algorithmic bytes, seconds, description)."""
+def oracle_decode_jobs(shapes, rows=None):
+    """The oracle's own packing of each decode shape's weight (rows: the first rows only)."""
     import oracle as O
-    try:
-        from threadpoolctl import threadpool_limits
-        limiter = threadpool_limits(limits=1)
-    except ImportError:  # pragma: no cover
-        limiter = None
-    total_bytes, total_t = 0, 0.0
+    jobs = []
     for (N, K) in shapes:
         W, mag, X = synth.decode_layer(N, K, 1)
         s = np.power(mag.astype(np.float64), 0.5).astype(np.float32)
-        Wr = W[:rows]
-        qw, sc, z = O.quantize_pack(Wr, s, 4, GROUP)
-        for _ in range(repeats):
-            t0 = time.perf_counter()
-            O.gemm_w4a16(X[:1], qw, sc, z, rows, K, 4, GROUP)
-            total_t += time.perf_counter() - t0
-            total_bytes += gemm_bytes(1, rows, K)
-    if limiter is not None:
-        limiter.unregister() if hasattr(limiter, "unregister") else None
-    desc = (f"oracle gemm_w4a16 (numpy fp64, 1 thread) at M=1 on the first {rows} rows of each "
-            f"decode shape, {repeats} calls each")
-    return total_bytes / total_t / 1e9, total_t, desc
+        Wr = W if rows is None else W[:rows]
+        jobs.append((X[:1], *O.quantize_pack(Wr, s, 4, GROUP), K, 4, GROUP))
+    return jobs
+
+
+def cpu_oracle_sample(shapes, min_seconds=10.0, max_seconds=30.0):
+    """The oracle (numpy, fp64) running the headline step -- the M = 1 decode GEMM over every
+    row of each decode shape -- on every host core (one spawned process per core, each on a
+    slice of the output rows), repeated for 10-30 s. Returns (GB/s of algorithmic bytes,
+    seconds, cores, description)."""
+    from oracle.parallel import OracleGemmPool, cpu_model
+    jobs = oracle_decode_jobs(shapes)
+    pool = OracleGemmPool(jobs)
+    try:
+        pool.run_once()   # warm-up
+        total, passes = 0.0, 0
+        while total < min_seconds and (passes == 0 or total + total / passes < max_seconds):
+            total += pool.run_once()
+            passes += 1
+    finally:
+        pool.close()
+    step_bytes = sum(gemm_bytes(1, qw.shape[0], K) for _, qw, _, _, K, _, _ in jobs)
+    desc = (f"oracle gemm_w4a16 (numpy fp64) at M=1 over all rows of {list(shapes)}, "
+            f"{passes} passes, output rows split across {pool.cores} spawned processes "
+            f"(1 BLAS thread each) on {cpu_model()}")
+    return step_bytes * passes / total / 1e9, total, pool.cores, desc
 
 
 # ----------------------------------------------------------------------------- other rows
@@ -331,18 +370,18 @@ def decoder_layer_rows(awq, dev, pk):
     ev[1].record()
     for xname, names in jobs:
         W = stacked[tuple(names)]
-        _, best, best_s, _ = awq.awq_search_scale(W, Xd[xname], stats[xname], alphas, 4,
-                                                  workspace=search_ws)
+        _, best, best_s, _, best_inv = awq.awq_search_scale(W, Xd[xname], stats[xname], alphas,
+                                                            4, workspace=search_ws, inv=True)
         search_flops += 20 * 2 * Xd[xname].shape[0] * W.shape[0] * W.shape[1]
         for n in names:
-            chosen[n] = (best, best_s)
+            chosen[n] = (best, best_s, best_inv)
     ev[2].record()
     packed = {n: awq.awq_quantize_pack(Wd[n], chosen[n][1], 4) for n in Wd}
     ev[3].record()
     gemm_flops = 0
     xin = {"q_proj": "hidden", "k_proj": "hidden", "v_proj": "hidden", "gate_proj": "hidden",
            "up_proj": "hidden", "o_proj": "o_in", "down_proj": "down_in"}
-    invs = {n: (1.0 / chosen[n][1]).contiguous() for n in packed}
+    invs = {n: chosen[n][2] for n in packed}
     ev3b = torch.cuda.Event(enable_timing=True)
     ev3b.record()
     for n, (qw, sc, z) in packed.items():
@@ -404,43 +443,41 @@ def profile_rows(awq, dev):
 # ----------------------------------------------------------------------------- main arms
 
 def run_reference(args, world, rank):
-    """The CPU oracle timed as the reference arm (rank 0 only)."""
+    """The CPU oracle timed as the reference arm (rank 0 only): each step is the headline
+    step (the M = 1 decode GEMM on the three decode shapes) on every host core, on all rows
+    when a pass takes under half a second, else on the first rows of each shape."""
     if rank != 0:
         return
-    import oracle as O
+    from oracle.parallel import OracleGemmPool, cpu_model
     shapes = synth.DECODE_SHAPES
-    rows = 256
-    prepared = []
-    for (N, K) in shapes:
-        W, mag, X = synth.decode_layer(N, K, 1)
-        s = np.power(mag.astype(np.float64), 0.5).astype(np.float32)
-        prepared.append((X[:1], O.quantize_pack(W[:rows], s, 4, GROUP), K))
+    rows = None
+    probe = OracleGemmPool(oracle_decode_jobs(shapes, rows=512))
+    t512 = min(probe.run_once() for _ in range(3))
+    probe.close()
+    full = sum(n for n, _ in shapes)
+    if t512 * full / (512 * len(shapes)) > 0.5:
+        rows = max(64, int(512 * 0.5 / t512))
+    jobs = oracle_decode_jobs(shapes, rows=rows)
+    pool = OracleGemmPool(jobs)
     try:
-        from threadpoolctl import threadpool_limits
-        threadpool_limits(limits=1)
-    except ImportError:  # pragma: no cover
-        pass
-    def step():
-        for X1, (qw, sc, z), K in prepared:
-            O.gemm_w4a16(X1, qw, sc, z, rows, K, 4, GROUP)
-    for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    dt = time.perf_counter() - t0
-    step_bytes = sum(gemm_bytes(1, rows, K) for _, _, K in prepared)
+        for _ in range(args.warmup):
+            pool.run_once()
+        dt = sum(pool.run_once() for _ in range(args.steps))
+    finally:
+        pool.close()
+    step_bytes = sum(gemm_bytes(1, qw.shape[0], K) for _, qw, _, _, K, _, _ in jobs)
     v = step_bytes * args.steps / dt / 1e9
-    sample = (f"each step: oracle gemm_w4a16 at M=1 on the first {rows} rows of each decode "
-              f"shape {shapes} (numpy fp64, 1 thread)")
+    sample = (f"each step: oracle gemm_w4a16 (numpy fp64) at M=1 on "
+              f"{'all rows' if rows is None else f'the first {rows} rows'} of each decode shape "
+              f"{shapes}, rows split across {pool.cores} spawned processes on {cpu_model()}")
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": "decode GEMM M=1 over [4096,4096], [11008,4096], [4096,11008] "
-                               "(W4 g128), row-sampled for the CPU oracle"},
-        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                               "(W4 g128), CPU oracle"},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": pool.cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -551,27 +588,30 @@ def run_b200(args, world, rank, local):
     prefill = []
     pf_cases = [(N, K, 4) for (N, K) in synth.PREFILL_SHAPES] + [(*synth.PREFILL_SHAPES[0], 3)]
     for (N, K, bits) in (pf_cases if args.only not in ("decode", "batched") else []):
-        W, mag, X = synth.prefill_layer(N, K, 2048)
+        m_list = synth.PREFILL_M if bits == 4 else [2048]
+        W, mag, X = synth.prefill_layer(N, K, max(m_list))
         s = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(dev)
         Wd = torch.from_numpy(W).to(dev)
         del W
         packs = [awq.awq_quantize_pack(Wd, s, bits)]
         del Wd
         packs.append(tuple(t.clone() for t in packs[0]))   # two copies > L2 with X
-        Xd = torch.from_numpy(X).to(dev)
-        Yd = torch.empty(2048, N, dtype=torch.float16, device=dev)
-        for p in packs:
-            awq.awq_gemm_w4a16(Xd, *p, N, K, bits, out=Yd)
-        torch.cuda.synchronize()
-        iters = 20
-        t = time_steps(lambda r: awq.awq_gemm_w4a16(Xd, *packs[r % 2], N, K, bits, out=Yd),
-                       iters, 3, stream, world)
-        tfl = 2 * 2048 * N * K * iters / t / 1e12
-        prefill.append({"N": N, "K": K, "M": 2048, "bits": bits, "ms": t / iters * 1e3,
-                        "TFLOP/s": tfl, "frac_tensor": tfl / pk["bf16_tflops"]})
-        del packs, Xd, Yd
+        Xall = torch.from_numpy(X).to(dev)
+        Yall = torch.empty(max(m_list), N, dtype=torch.float16, device=dev)
+        for M in m_list:
+            Xd, Yd = Xall[:M], Yall[:M]
+            for p in packs:
+                awq.awq_gemm_w4a16(Xd, *p, N, K, bits, out=Yd)
+            torch.cuda.synchronize()
+            iters = max(5, 20 * 2048 // M)
+            t = time_steps(lambda r: awq.awq_gemm_w4a16(Xd, *packs[r % 2], N, K, bits, out=Yd),
+                           iters, 3, stream, world)
+            tfl = 2 * M * N * K * iters / t / 1e12
+            prefill.append({"N": N, "K": K, "M": M, "bits": bits, "ms": t / iters * 1e3,
+                            "TFLOP/s": tfl, "frac_tensor": tfl / pk["bf16_tflops"]})
+        del packs, Xall, Yall
         torch.cuda.empty_cache()
-    pf4 = [p for p in prefill if p["bits"] == 4]
+    pf4 = [p for p in prefill if p["bits"] == 4 and p["M"] == 2048]
     pf_flops = sum(2 * 2048 * p["N"] * p["K"] for p in pf4)
     pf_time = sum(p["ms"] for p in pf4) / 1e3
     pf_value = pf_flops / pf_time / 1e12 if pf4 else None
@@ -580,8 +620,11 @@ def run_b200(args, world, rank, local):
 
     if rank != 0:
         return
-    cpu_gbs, cpu_t, cpu_desc = (cpu_oracle_sample(synth.DECODE_SHAPES) if args.only == "all"
-                                else (None, None, "skipped (--only)"))
+    cpu_gbs, cpu_t, cpu_cores, cpu_desc = (cpu_oracle_sample(synth.DECODE_SHAPES)
+                                           if args.only == "all"
+                                           else (None, None, None, "skipped (--only)"))
+    dec_traffic, dec_traffic_src = profiled_traffic("gemv_stream_decode_M1")
+    pf_traffic, pf_traffic_src = profiled_traffic("tc_gemm_prefill_28672x8192_M2048")
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt_max / args.steps * 1e3,
@@ -593,26 +636,28 @@ def run_b200(args, world, rank, local):
             "inputs": "weights rotate through copies totalling > 2x L2 (L2 not flushed)",
             "replay": "warm-up steps and the K timed steps each captured in one CUDA graph "
                       "(kernels back to back, programmatic dependent launch between them)",
+            "flags": "AWQ_GEMM_WEIGHTS_READY (static weights: each GEMM streams its weights "
+                     "while the previous GEMM runs; activations are read after it completes)",
             "parallelism": f"replicas x{world} (no data-path collective)",
         },
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": pk["hbm_gbs"],
                      "unit": "GB/s", "frac": per_gpu / pk["hbm_gbs"],
-                     "traffic": DECODE_TRAFFIC_PER_LAUNCH,
+                     "traffic": dec_traffic, "traffic_source": dec_traffic_src,
                      "algorithmic_bytes_per_launch": step_bytes / len(synth.DECODE_SHAPES),
-                     "kernel": "gemv_stream_kernel<1, true>", "peak_source": pk["source"],
+                     "kernel": "gemv_stream_kernel<1, true, 8>", "peak_source": pk["source"],
                      "peak_kind": "measured copy bandwidth (burst)",
                      "frac_of_8TBps_nominal": per_gpu / 8000.0},
         "prefill": {"metric": "TFLOP/s at M=2048", "value": pf_value, "unit": "TFLOP/s",
                     "per_shape": prefill, "peak": pk["bf16_tflops"],
                     "peak_kind": "measured bf16 cuBLAS burst (fp16 has the same dense rate)",
-                    "traffic_28672x8192": PREFILL_TRAFFIC_PER_LAUNCH,
+                    "traffic_28672x8192": pf_traffic, "traffic_source": pf_traffic_src,
                     "frac": pf_value / pk["bf16_tflops"] if prefill else None,
                     "kernel": "tc_gemm_kernel"},
         "sweep": sweep,
         "batched": batched,
         "rows": rows,
-        "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": cpu_desc, "seconds": cpu_t},
+        "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": cpu_cores,
+                         "kind": "oracle", "sample": cpu_desc, "seconds": cpu_t},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk,

@@ -63,7 +63,8 @@ typedef enum {
   AWQ_ERR_UNSUPPORTED = 2,   /* valid request the library does not implement */
   AWQ_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the size query's answer */
   AWQ_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (e.g. no GPU, launch) */
-  AWQ_ERR_TIMEOUT = 5        /* a kernel's bounded wait ran out (see awq_check_error) */
+  AWQ_ERR_TIMEOUT = 5,       /* a kernel's bounded wait ran out (see awq_check_error) */
+  AWQ_ERR_BOUNDS = 6         /* debug build only: a kernel's index check failed */
 } awq_status;
 
 /* Human-readable name of a status code. Never NULL. */
@@ -73,8 +74,9 @@ AWQ_API const char* awq_status_string(awq_status status);
 AWQ_API int awq_abi_version(void);
 
 /* Synchronises `stream`, then reads and clears the device status word of the current
- * device. Returns AWQ_ERR_TIMEOUT if a kernel reported a bounded-wait timeout since the
- * last check, AWQ_ERR_CUDA if the synchronisation failed, AWQ_OK otherwise. */
+ * device. Returns AWQ_ERR_BOUNDS if (in the debug build) a kernel's index check failed,
+ * else AWQ_ERR_TIMEOUT if a kernel reported a bounded-wait timeout since the last check,
+ * AWQ_ERR_CUDA if the synchronisation failed, AWQ_OK otherwise. */
 AWQ_API awq_status awq_check_error(void* stream);
 
 /* Self-test of failure detection: launches one thread that waits on a barrier nothing ever
@@ -83,6 +85,15 @@ AWQ_API awq_status awq_check_error(void* stream);
  * wait ran out, sets the device status word, and returns; the next awq_check_error() on
  * the stream returns AWQ_ERR_TIMEOUT and the context stays usable. */
 AWQ_API awq_status awq_selftest_timeout(int* waited_out, void* stream);
+
+/* Self-test of the debug build's bounds checks (libawq_b200_debug.so, compiled with
+ * AWQ_DEBUG_BOUNDS; in that build every kernel checks the indices of its global and shared
+ * memory accesses against the extents the call's shapes give, skips an access that falls
+ * outside, and records it in the device status word). Launches one thread that stores
+ * buf[i] = i for i = 0..4 into a device buffer of 4 ints (16-byte aligned): the check stops
+ * the fifth store, so buf holds 0..3 and the next awq_check_error() returns AWQ_ERR_BOUNDS.
+ * The release build has no checks and returns AWQ_ERR_UNSUPPORTED without launching. */
+AWQ_API awq_status awq_selftest_bounds(int* buf, void* stream);
 
 /* ---------------------------------------------------------------- activation statistics
  * robotsatlas.com "AWQ", "How it works" / "Components: Activation saliency analysis":
@@ -143,32 +154,48 @@ AWQ_API awq_status awq_quantize_pack(const awq_f16* W, int64_t N, int64_t K, con
  * W: fp16 [N, K]; X: fp16 [M, K] (calibration tokens); s_x: fp32 [K]; alphas: fp32 device
  * array [n_alpha] (1 <= n_alpha <= 64); s_table: NULL or fp32 [n_alpha, K].
  * Outputs (device): losses fp64 [n_alpha], best_idx int32 [1], best_s fp32 [K],
- * row_losses NULL or fp64 [n_alpha, N] (each row's share of L[a]).
+ * best_inv_s NULL or fp32 [K] (1 / best_s, correctly rounded: the inv_s that
+ * awq_gemm_w4a16 takes for a layer packed with best_s), row_losses NULL or fp64
+ * [n_alpha, N] (each row's share of L[a]).
  * workspace: at least awq_search_scale_workspace_size(M, N, K, n_alpha) bytes. */
 AWQ_API size_t awq_search_scale_workspace_size(int64_t M, int64_t N, int64_t K, int n_alpha);
 AWQ_API awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f16* X,
                             int64_t M, const float* s_x, const float* alphas, int n_alpha,
                             int bits, int group, const float* s_table, double* losses,
-                            int32_t* best_idx, float* best_s, double* row_losses,
-                            void* workspace, size_t ws_bytes, void* stream);
+                            int32_t* best_idx, float* best_s, float* best_inv_s,
+                            double* row_losses, void* workspace, size_t ws_bytes,
+                            void* stream);
 
 /* ---------------------------------------------------------------- W4A16 GEMM
  * builderai.tools "AWQ", "About" (kernels for 4-bit weights with 16-bit activations);
  * robotsatlas.com "AWQ", "Implementation pitfalls" (dequantization fused into the GEMM).
- *     Y[m, n] = sum_k x'[m, k] * (q[n, k] - z[k/128, n]) * scale[k/128, n]
- * with x' = X, or x' = fp16(X[m, k] * inv_s[k]) when inv_s is not NULL (the activation side
- * of the per-channel scaling). fp32 accumulation, fp16 output.
+ *     Y[m, n] = sum_k X[m, k] * inv_s[k] * (q[n, k] - z[k/128, n]) * scale[k/128, n]
+ * with inv_s[k] = 1 when inv_s is NULL (inv_s is the activation side of the per-channel
+ * scaling: 1/s for a layer packed with W diag(s)). fp32 accumulation, fp16 output. The
+ * decode kernels apply inv_s to the activations in fp32 (x' = fp16(x * inv_s)); the
+ * tensor-core kernel folds it into the dequantized weights (fp16(scale * inv_s[k]) per k),
+ * so no extra pass over X is made.
  * M <= 16 with 4 bits runs a decode kernel (HBM-bound GEMV; for 8 < M <= 16 only when X
  * fits in one CTA's shared memory); other calls (and 3 bits) run the tensor-core kernel.
  * X: fp16 [M, K]; Y: fp16 [M, N]. M = 0 or N = 0 is a no-op.
- * workspace: at least awq_gemm_workspace_size(M, N, K, bits) bytes: 0 for the decode
- * kernels, otherwise room for x' and, when K is split across CTAs, the fp32 partial sums
- * (the size does not depend on whether inv_s is given). */
+ * flags: 0, or AWQ_GEMM_WEIGHTS_READY. The kernels are launched with programmatic dependent
+ * launch, so a kernel of this call may start while the kernel launched just before it on
+ * `stream` is still running; by default it reads nothing before that kernel has completed.
+ * AWQ_GEMM_WEIGHTS_READY states that qweight, scales and zeros are NOT written by the kernel
+ * launched immediately before this call on `stream` (they were written earlier, e.g. model
+ * weights loaded once): the decode kernel then starts streaming them at once, overlapping
+ * the preceding kernel. X is always read only after the preceding kernel has completed.
+ * (This library's kernels let the next launch start only after their own predecessor has
+ * completed, so with them the window is exactly one kernel.) Other bits are rejected.
+ * workspace: at least awq_gemm_workspace_size(M, N, K, bits) bytes: 0 unless the
+ * tensor-core kernel splits K across CTAs (few output tiles), then room for the fp32
+ * partial sums; the size does not depend on inv_s or flags. */
+#define AWQ_GEMM_WEIGHTS_READY 1u
 AWQ_API size_t awq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits);
 AWQ_API awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
                           const awq_f16* scales, const uint8_t* zeros, int64_t N, int64_t K,
-                          int bits, int group, const float* inv_s, awq_f16* Y, void* workspace,
-                          size_t ws_bytes, void* stream);
+                          int bits, int group, const float* inv_s, unsigned flags, awq_f16* Y,
+                          void* workspace, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

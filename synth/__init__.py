@@ -154,18 +154,19 @@ def decoder_layer_weights(hidden: int = 4096, mlp: int = 11008):
 
 
 def decoder_layer_activations(tokens: int = 128 * 512, hidden: int = 4096, mlp: int = 11008,
-                              names=("hidden", "o_in", "down_in")):
+                              names=("hidden", "o_in", "down_in"), rows: int | None = None):
     """Seed 4: the layer's three calibration inputs of ``tokens`` rows, each N(0, 1) times its
     own lognormal(0, 0.7) channel magnitudes with round(0.01 K) outlier channels multiplied
     by U(10, 50): the hidden state X (input of q/k/v and gate/up), X_o (input of o_proj) and
     X_d (input of down_proj). Each input has its own stream (SeedSequence [4, tokens, K, i],
     i = 0, 1, 2 in that order), drawing magnitudes, outlier indices, gains, then X, so any
-    subset can be generated alone."""
+    subset can be generated alone. ``rows`` draws only the first rows of the same inputs
+    (normal draws fill row by row, so they are exactly the leading rows of the full batch)."""
     dims = {"hidden": (0, hidden), "o_in": (1, hidden), "down_in": (2, mlp)}
     out = {}
     for name in names:
         idx, k = dims[name]
         rng = _rng(4, tokens, k, idx)
         m = channel_magnitudes(rng, k, 0.7, outlier_gain=(10.0, 50.0))
-        out[name] = random_activations(rng, tokens, m)
+        out[name] = random_activations(rng, tokens if rows is None else rows, m)
     return out

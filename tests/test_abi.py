@@ -43,9 +43,10 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_version():
     L = _lib()
     for code, name in enumerate(["AWQ_OK", "AWQ_ERR_INVALID_ARG", "AWQ_ERR_UNSUPPORTED",
-                                 "AWQ_ERR_WORKSPACE", "AWQ_ERR_CUDA", "AWQ_ERR_TIMEOUT"]):
+                                 "AWQ_ERR_WORKSPACE", "AWQ_ERR_CUDA", "AWQ_ERR_TIMEOUT",
+                                 "AWQ_ERR_BOUNDS"]):
         assert L.awq_status_string(code).decode() == name
-    assert L.awq_abi_version() == 1
+    assert L.awq_abi_version() == 2
 
 
 def test_host_validation_rejects_before_launch():
@@ -64,26 +65,32 @@ def test_host_validation_rejects_before_launch():
     assert L.awq_quantize_pack(fake, 4, 200, None, 4, 128, fake, fake, fake, None) == 1
     assert L.awq_quantize_pack(fake, 0, 128, None, 4, 128, fake, fake, fake, None) == 0
     # gemm: M = 0 and N = 0 are no-ops; misaligned Y; bits 2
-    assert L.awq_gemm_w4a16(fake, 0, fake, fake, fake, 8, 128, 4, 128, None, fake, None, 0,
+    assert L.awq_gemm_w4a16(fake, 0, fake, fake, fake, 8, 128, 4, 128, None, 0, fake, None, 0,
                             None) == 0
-    assert L.awq_gemm_w4a16(fake, 1, fake, fake, fake, 0, 128, 4, 128, None, fake, None, 0,
+    assert L.awq_gemm_w4a16(fake, 1, fake, fake, fake, 0, 128, 4, 128, None, 0, fake, None, 0,
                             None) == 0
-    assert L.awq_gemm_w4a16(fake, 1, fake, fake, fake, 8, 128, 4, 128, None, odd, None, 0,
+    assert L.awq_gemm_w4a16(fake, 1, fake, fake, fake, 8, 128, 4, 128, None, 0, odd, None, 0,
                             None) == 1
-    assert L.awq_gemm_w4a16(fake, 1, fake, fake, fake, 8, 128, 2, 128, None, fake, None, 0,
+    assert L.awq_gemm_w4a16(fake, 1, fake, fake, fake, 8, 128, 2, 128, None, 0, fake, None, 0,
+                            None) == 1
+    # unknown flag bits
+    assert L.awq_gemm_w4a16(fake, 1, fake, fake, fake, 8, 128, 4, 128, None, 6, fake, None, 0,
                             None) == 1
     # search: n_alpha out of range, too-small workspace
     assert L.awq_search_scale(fake, 8, 128, fake, 4, fake, fake, 0, 4, 128, None, fake, fake,
-                              fake, None, fake, 1 << 30, None) == 1
+                              fake, None, None, fake, 1 << 30, None) == 1
     assert L.awq_search_scale(fake, 8, 128, fake, 4, fake, fake, 20, 4, 128, None, fake, fake,
-                              fake, None, fake, 16, None) == 3
+                              fake, None, None, fake, 16, None) == 3
+    assert L.awq_search_scale(fake, 8, 128, fake, 4, fake, fake, 20, 4, 128, None, fake, fake,
+                              fake, odd, None, fake, 1 << 30, None) == 1
 
 
 def test_workspace_queries():
     L = _lib()
     assert L.awq_search_scale_workspace_size(256, 512, 512, 20) >= 20 * 512 * 512 * 2
     assert L.awq_gemm_workspace_size(1, 4096, 4096, 4) == 0
-    assert L.awq_gemm_workspace_size(2048, 4096, 4096, 4) >= 2048 * 4096 * 2
+    # enough output tiles for every SM: no split-K, no workspace (inv_s needs none)
+    assert L.awq_gemm_workspace_size(2048, 4096, 4096, 4) == 0
     assert L.awq_act_stats_workspace_size(0, 16) == 0
 
 
@@ -97,25 +104,39 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
 
 def test_gemm_workspace_follows_the_chosen_kernel():
     # the decode kernels need no workspace; an 8 < M <= 16 call whose X does not fit the
-    # streaming kernel's shared memory takes the tensor-core path and needs room for x'
+    # streaming kernel's shared memory takes the tensor-core path, which with so few output
+    # tiles splits K and needs room for fp32 partial sums (at least two slices of M x N)
     L = _lib()
     assert L.awq_gemm_workspace_size(1, 4096, 11008, 4) == 0
     assert L.awq_gemm_workspace_size(8, 4096, 11008, 4) == 0
     assert L.awq_gemm_workspace_size(16, 4096, 4096, 4) == 0
-    assert L.awq_gemm_workspace_size(16, 4096, 11008, 4) >= 16 * 11008 * 2
-    assert L.awq_gemm_workspace_size(16, 4104, 4096, 4) >= 16 * 4096 * 2   # N % 16 != 0
-    assert L.awq_gemm_workspace_size(64, 4096, 4096, 4) >= 64 * 4096 * 2
+    for M, N, K in [(16, 4096, 11008), (16, 4104, 4096), (64, 4096, 4096)]:  # 4104: N % 16
+        ws = L.awq_gemm_workspace_size(M, N, K, 4)
+        assert ws >= 2 * M * N * 4 and ws % 256 == 0, (M, N, K, ws)
 
 
 def test_gemm_workspace_is_checked_before_launch():
-    # the tensor-core path with inv_s needs room for x'; a missing or short workspace is
-    # rejected on the host (AWQ_ERR_WORKSPACE) before anything is launched
+    # the tensor-core path with few output tiles needs room for split-K partial sums; a
+    # missing or short workspace is rejected on the host (AWQ_ERR_WORKSPACE) before anything
+    # is launched
     L = _lib()
     P = ctypes.c_void_p
     fake = P(1 << 20)
     need = L.awq_gemm_workspace_size(64, 4096, 4096, 4)
-    assert need >= 64 * 4096 * 2
-    assert L.awq_gemm_w4a16(fake, 64, fake, fake, fake, 4096, 4096, 4, 128, fake, fake, None,
-                            0, None) == 3
-    assert L.awq_gemm_w4a16(fake, 64, fake, fake, fake, 4096, 4096, 4, 128, fake, fake, fake,
-                            64 * 4096 * 2 - 16, None) == 3
+    assert need >= 2 * 64 * 4096 * 4
+    assert L.awq_gemm_w4a16(fake, 64, fake, fake, fake, 4096, 4096, 4, 128, fake, 0, fake,
+                            None, 0, None) == 3
+    assert L.awq_gemm_w4a16(fake, 64, fake, fake, fake, 4096, 4096, 4, 128, fake, 0, fake,
+                            fake, need - 16, None) == 3
+
+
+def test_debug_build_exports_the_same_symbols():
+    # the bounds-checking build is the same library with index checks compiled in
+    from weight_only_int4_stats_b200 import build
+    import weight_only_int4_stats_b200 as awq
+    D = awq.load_library(build.build(debug=True))
+    for name in _declared():
+        assert hasattr(D, name), name
+    assert D.awq_abi_version() == 2
+    # the release build refuses the bounds self-test without launching anything
+    assert _lib().awq_selftest_bounds(ctypes.c_void_p(1 << 20), None) == 2

@@ -25,6 +25,10 @@ pytestmark = pytest.mark.gpu
 GEMM_RTOL = 2e-3
 LOSS_RTOL = 2.0 ** -10
 NEAR_TIE = 2.0 ** -10
+# On the 512 x 512 seed-0 layer (256 tokens, 512 rows) the fp16 rounding of E averages out
+# and the losses agree to ~1e-6, so there the chosen grid point may differ from the oracle's
+# only when the oracle rates the two within 1e-5 of each other.
+NEAR_TIE_SINGLE_LAYER = 1e-5
 
 
 @pytest.fixture(scope="module")
@@ -152,6 +156,22 @@ def test_gemm_decode_inv_s(awq, M):
     _check_gemm(awq, X, qw, sc, z, N, K, inv_s=inv_s)
 
 
+@pytest.mark.parametrize("with_inv_s", [False, True])
+def test_gemm_decode_outlier_activations_k11008(awq, with_inv_s):
+    # down_proj-shaped decode ([4096, 11008]) on tokens of the 7B-shaped layer's down_proj
+    # calibration input (lognormal(0, 0.7) magnitudes, 1% of channels x U(10, 50)): at M = 1
+    # the kernel removes a 1024 offset per group with fp32 activation sums, which these large
+    # activations stress. The weight is quantized with s = s_x^0.5 of those activations.
+    X = synth.decoder_layer_activations(names=("down_in",), rows=16)["down_in"]
+    W = synth.decoder_layer_weights()["down_proj"]
+    N, K = W.shape
+    s = O.scale_candidates(O.act_stats(X), np.array([0.5], np.float32))[0]
+    qw, sc, z = _packed(W, s)
+    inv = (1.0 / s).astype(np.float32) if with_inv_s else None
+    for M in (1, 4, 16):
+        _check_gemm(awq, X[:M], qw, sc, z, N, K, inv_s=inv)
+
+
 @pytest.mark.parametrize("N,K", synth.DECODE_SHAPES)
 def test_gemm_decode_full_shapes(awq, N, K):
     W, m, X = synth.decode_layer(N, K)
@@ -199,12 +219,16 @@ def test_gemm_3bit_decode_sizes(awq, M):
     _check_gemm(awq, X, qw, sc, z, N, K, 3)
 
 
-def test_gemm_tensor_core_inv_s(awq):
-    N, K, M = 256, 512, 96
-    W, X, m = rand_layer(77, N, K, M)
+@pytest.mark.parametrize("bits", [4, 3])
+@pytest.mark.parametrize("M,N,K", [(17, 256, 512), (32, 384, 1024), (96, 256, 512),
+                                   (2048, 1024, 2048)])
+def test_gemm_tensor_core_inv_s(awq, M, N, K, bits):
+    # inv_s on the tensor-core path is folded into the dequantized weights (one combined
+    # fp16 scale per k), with and without split-K
+    W, X, m = rand_layer(77 + M + bits, N, K, M)
     s = np.sqrt(m).astype(np.float32)
-    qw, sc, z = _packed(W, s)
-    _check_gemm(awq, X, qw, sc, z, N, K, inv_s=(1.0 / s).astype(np.float32))
+    qw, sc, z = _packed(W, s, bits)
+    _check_gemm(awq, X, qw, sc, z, N, K, bits, inv_s=(np.float32(1.0) / s).astype(np.float32))
 
 
 @pytest.mark.parametrize("N,K", synth.BATCHED_SHAPES)
@@ -219,21 +243,29 @@ def test_gemm_batched_full_shapes(awq, N, K):
 @pytest.mark.parametrize("N,K,bits", [(n, k, 4) for (n, k) in synth.PREFILL_SHAPES] +
                          [(synth.PREFILL_SHAPES[0][0], synth.PREFILL_SHAPES[0][1], 3)])
 def test_gemm_prefill_full_shape_sampled(awq, N, K, bits):
-    # Full-size launch (M = 2048); the oracle checks 16 sampled token rows against all N.
-    W, m, X = synth.prefill_layer(N, K, 2048)
-    qw, sc, z = _packed(W, np.power(m.astype(np.float64), 0.5).astype(np.float32), bits)
-    rows = np.random.default_rng(0).choice(2048, 16, replace=False)
-    rows.sort()
-    _check_gemm(awq, X, qw, sc, z, N, K, bits, rows=rows)
-    torch.cuda.empty_cache()
+    # Full-size launches at M = 2048, 4096 and 8192 (M = 2048 only for the 3-bit variant);
+    # the oracle checks 16 sampled token rows against all N. The GPU's own quantize-and-pack
+    # of the weight must equal the oracle's bit for bit.
+    W, m, X = synth.prefill_layer(N, K, synth.PREFILL_M[-1] if bits == 4 else 2048)
+    s = np.power(m.astype(np.float64), 0.5).astype(np.float32)
+    qw, sc, z = _packed(W, s, bits)
+    gq, gs, gz = awq.awq_quantize_pack(cu(W), cu(s), bits)
+    np.testing.assert_array_equal(host_u32(gq), qw)
+    np.testing.assert_array_equal(gs.cpu().numpy().view(np.uint16), sc.view(np.uint16))
+    np.testing.assert_array_equal(gz.cpu().numpy(), z)
+    del gq, gs, gz, W
+    for M in (synth.PREFILL_M if bits == 4 else [2048]):
+        rows = np.sort(np.random.default_rng(M).choice(M, 16, replace=False))
+        _check_gemm(awq, X[:M], qw, sc, z, N, K, bits, rows=rows)
+        torch.cuda.empty_cache()
 
 
 # ----------------------------------------------------------------------------- search
 
-def _alpha_parity(gpu_best, ora_losses):
+def _alpha_parity(gpu_best, ora_losses, near_tie=NEAR_TIE):
     ob = int(np.argmin(ora_losses))
     if gpu_best != ob:
-        assert ora_losses[gpu_best] <= (1 + NEAR_TIE) * ora_losses[ob], (gpu_best, ob)
+        assert ora_losses[gpu_best] <= (1 + near_tie) * ora_losses[ob], (gpu_best, ob)
 
 
 @pytest.mark.parametrize("bits", [4, 3])
@@ -246,7 +278,7 @@ def test_search_single_layer_same_scales(awq, bits):
     ol = O.search_losses(W, X, None, a, bits, 128, s_table=table)
     np.testing.assert_allclose(losses.cpu().numpy(), ol, rtol=LOSS_RTOL)
     b = int(best.item())
-    _alpha_parity(b, ol)
+    _alpha_parity(b, ol, NEAR_TIE_SINGLE_LAYER)
     np.testing.assert_array_equal(best_s.cpu().numpy(), table[b])
     orow = O.search_losses(W, X, None, a, bits, 128, s_table=table, per_row=True)
     np.testing.assert_allclose(rows.cpu().numpy(), orow, rtol=1e-3, atol=1e-12 * orow.max())
@@ -263,7 +295,7 @@ def test_search_single_layer_pipeline(awq):
     np.testing.assert_array_equal(s_x.cpu().numpy(), O.act_stats(X))
     np.testing.assert_allclose(losses.cpu().numpy(), ol, rtol=LOSS_RTOL)
     b = int(best.item())
-    _alpha_parity(b, ol)
+    _alpha_parity(b, ol, NEAR_TIE_SINGLE_LAYER)
     gs = best_s.cpu().numpy()
     if b == ob:
         np.testing.assert_allclose(gs, obs, rtol=2 ** -23)   # fp64 pow on both sides
@@ -290,26 +322,48 @@ def test_search_small_and_ragged(awq, N, K, M, bits):
     _alpha_parity(int(best.item()), ol)
 
 
-def test_search_joint_equals_sum_of_parts(awq):
+def test_search_joint_against_oracle(awq):
+    # q/k/v-style joint search: three weights sharing one input, searched as their
+    # row-concatenation; the GPU's losses and grid index against the oracle's search of the
+    # same concatenated weight, and each part's share of the per-row losses against the
+    # oracle's search of that part alone.
     rng = np.random.default_rng(3)
     parts = [(rng.standard_normal((n, 256), dtype=np.float32) * 0.02).astype(np.float16)
              for n in (96, 64, 160)]
     _, X, _ = rand_layer(4, 1, 256, 64)
-    a = cu(O.alpha_grid(20))
+    a = O.alpha_grid(20)
+    Wj = np.concatenate(parts)
     s_x = awq.awq_act_stats(cu(X))
-    joint, *_ = awq.awq_search_scale(cu(np.concatenate(parts)), cu(X), s_x, a, 4)
-    each = sum(awq.awq_search_scale(cu(p), cu(X), s_x, a, 4)[0] for p in parts)
-    np.testing.assert_allclose(joint.cpu().numpy(), each.cpu().numpy(), rtol=1e-9)
+    losses, best, best_s, rows = awq.awq_search_scale(cu(Wj), cu(X), s_x, cu(a), 4,
+                                                      row_losses=True)
+    o_sx = O.act_stats(X)
+    ol, ob, obs = O.search_scale(Wj, X, o_sx, a, 4, 128)
+    np.testing.assert_allclose(losses.cpu().numpy(), ol, rtol=LOSS_RTOL)
+    _alpha_parity(int(best.item()), ol)
+    rows = rows.cpu().numpy()
+    off = 0
+    for p in parts:
+        op = O.search_losses(p, X, o_sx, a, 4, 128)
+        np.testing.assert_allclose(rows[:, off:off + p.shape[0]].sum(axis=1), op, rtol=LOSS_RTOL)
+        off += p.shape[0]
 
 
-def test_search_full_decoder_layer_sampled_rows(awq):
-    # Full-size joint gate/up search (N = 22016, K = 4096, M = 65536): the oracle recomputes
-    # the per-row losses of 8 sampled rows; the grid index is checked through those rows'
-    # share only as a consistency check (the full argmin needs every row).
-    acts = synth.decoder_layer_activations()
+@pytest.mark.parametrize("job", ["qkv", "gate_up", "o_proj", "down_proj"])
+def test_search_full_decoder_layer_sampled_rows(awq, job):
+    # Each of the 7B-shaped layer's four searches at full size (65536 calibration tokens; q/k/v
+    # jointly with N = 12288, gate/up jointly with N = 22016, o_proj, and down_proj with
+    # K = 11008): the oracle recomputes the per-row losses of 8 sampled rows at every grid
+    # point, and the per-row losses must add up to the reported totals. The argmin over all
+    # rows is checked against the oracle on the same layer at 1024 tokens
+    # (tests/test_gpu_pipeline.py), where the oracle can evaluate every row.
+    xname, names = {"qkv": ("hidden", ["q_proj", "k_proj", "v_proj"]),
+                    "gate_up": ("hidden", ["gate_proj", "up_proj"]),
+                    "o_proj": ("o_in", ["o_proj"]),
+                    "down_proj": ("down_in", ["down_proj"])}[job]
+    X = synth.decoder_layer_activations(names=(xname,))[xname]
     Wd = synth.decoder_layer_weights()
-    X = acts["hidden"]
-    W = np.concatenate([Wd["gate_proj"], Wd["up_proj"]])
+    W = np.concatenate([Wd[n] for n in names])
+    del Wd
     a = O.alpha_grid(20)
     table = O.scale_candidates(O.act_stats(X), a)
     losses, best, best_s, rows = awq.awq_search_scale(cu(W), cu(X), None, None, 4,
@@ -322,7 +376,7 @@ def test_search_full_decoder_layer_sampled_rows(awq):
     b = int(best.item())
     assert b == int(np.argmin(losses.cpu().numpy()))
     np.testing.assert_array_equal(best_s.cpu().numpy(), table[b])
-    del acts, X
+    del X
     torch.cuda.empty_cache()
 
 
@@ -359,6 +413,29 @@ def test_decode_chain_output_feeds_next_input(awq):
     o1 = O.gemm_w4a16(X, *p1, N1, K1, 4, 128).astype(np.float16)
     o2 = O.gemm_w4a16(o1, *p2, N2, N1, 4, 128)
     assert rel_fro(Y2.float().cpu().numpy(), o2) <= GEMM_RTOL
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_chain_weights_ready(awq, M):
+    # AWQ_GEMM_WEIGHTS_READY: each call starts streaming its (static) packed weights while the
+    # previous GEMM on the stream still runs; its activations are that GEMM's output. Three
+    # back-to-back decode GEMMs (shapes of o_proj, up_proj, down_proj), twice in a row.
+    shapes = [(4096, 4096), (11008, 4096), (4096, 11008)]
+    rng = np.random.default_rng(31 + M)
+    Ws = [(rng.standard_normal((n, k), dtype=np.float32) * 0.02).astype(np.float16)
+          for n, k in shapes]
+    packs = [O.quantize_pack(W, None, 4, 128) for W in Ws]
+    dev = [[cu(a) for a in p] for p in packs]
+    X = (rng.standard_normal((M, 4096), dtype=np.float32)).astype(np.float16)
+    for _ in range(2):
+        h = cu(X)
+        for (n, k), d in zip(shapes, dev):
+            h = awq.awq_gemm_w4a16(h, *d, n, k, weights_ready=True)
+    got = h.float().cpu().numpy()
+    want = X
+    for (n, k), p in zip(shapes, packs):
+        want = O.gemm_w4a16(want, *p, n, k, 4, 128).astype(np.float16)
+    assert rel_fro(got, want.astype(np.float64)) <= GEMM_RTOL
 
 
 @pytest.mark.parametrize("M,N,K", [(64, 1024, 1024), (64, 1000, 1024), (40, 512, 2304),

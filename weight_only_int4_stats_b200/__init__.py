@@ -13,9 +13,9 @@ import os
 import torch
 
 __all__ = [
-    "AwqError", "lib", "library_path", "GROUP",
+    "AwqError", "lib", "load_library", "library_path", "GROUP",
     "awq_act_stats", "awq_act_stats_noalloc", "awq_quantize_pack", "awq_search_scale", "awq_gemm_w4a16",
-    "awq_check_error", "packed_words_per_row",
+    "awq_check_error", "packed_words_per_row", "WEIGHTS_READY",
 ]
 
 GROUP = 128
@@ -23,7 +23,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libawq_b200.so")
 
 STATUS = {0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_UNSUPPORTED",
-          3: "AWQ_ERR_WORKSPACE", 4: "AWQ_ERR_CUDA", 5: "AWQ_ERR_TIMEOUT"}
+          3: "AWQ_ERR_WORKSPACE", 4: "AWQ_ERR_CUDA", 5: "AWQ_ERR_TIMEOUT", 6: "AWQ_ERR_BOUNDS"}
 
 
 class AwqError(RuntimeError):
@@ -36,36 +36,44 @@ class AwqError(RuntimeError):
 _lib = None
 
 
+def load_library(path: str) -> ctypes.CDLL:
+    """Loads a build of the library (the release build, or the bounds-checking debug build)
+    and declares every entry point's signature. Raises ImportError if it is missing."""
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with "
+            "`python -m weight_only_int4_stats_b200.build` (there is no CPU fallback)")
+    L = ctypes.CDLL(path)
+    P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "awq_status_string": (ctypes.c_char_p, [I32]),
+        "awq_abi_version": (I32, []),
+        "awq_check_error": (I32, [P]),
+        "awq_selftest_timeout": (I32, [P, P]),
+        "awq_selftest_bounds": (I32, [P, P]),
+        "awq_act_stats_workspace_size": (SZ, [I64, I64]),
+        "awq_act_stats": (I32, [P, I64, I64, P, P, SZ, P]),
+        "awq_act_stats_noalloc": (I32, [P, I64, I64, P, P]),
+        "awq_quantize_pack": (I32, [P, I64, I64, P, I32, I32, P, P, P, P]),
+        "awq_search_scale_workspace_size": (SZ, [I64, I64, I64, I32]),
+        "awq_search_scale": (I32, [P, I64, I64, P, I64, P, P, I32, I32, I32, P, P, P, P, P,
+                                   P, P, SZ, P]),
+        "awq_gemm_workspace_size": (SZ, [I64, I64, I64, I32]),
+        "awq_gemm_w4a16": (I32, [P, I64, P, P, P, I64, I64, I32, I32, P, ctypes.c_uint, P,
+                                 P, SZ, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
 def lib() -> ctypes.CDLL:
     """The loaded CUDA library (loaded on first use; raises if it was never built)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(library_path):
-            raise ImportError(
-                f"{library_path} is missing: build it with "
-                "`python -m weight_only_int4_stats_b200.build` (there is no CPU fallback)")
-        L = ctypes.CDLL(library_path)
-        P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
-        sig = {
-            "awq_status_string": (ctypes.c_char_p, [I32]),
-            "awq_abi_version": (I32, []),
-            "awq_check_error": (I32, [P]),
-            "awq_selftest_timeout": (I32, [P, P]),
-            "awq_act_stats_workspace_size": (SZ, [I64, I64]),
-            "awq_act_stats": (I32, [P, I64, I64, P, P, SZ, P]),
-            "awq_act_stats_noalloc": (I32, [P, I64, I64, P, P]),
-            "awq_quantize_pack": (I32, [P, I64, I64, P, I32, I32, P, P, P, P]),
-            "awq_search_scale_workspace_size": (SZ, [I64, I64, I64, I32]),
-            "awq_search_scale": (I32, [P, I64, I64, P, I64, P, P, I32, I32, I32, P, P, P, P, P,
-                                       P, SZ, P]),
-            "awq_gemm_workspace_size": (SZ, [I64, I64, I64, I32]),
-            "awq_gemm_w4a16": (I32, [P, I64, P, P, P, I64, I64, I32, I32, P, P, P, SZ, P]),
-        }
-        for name, (res, args) in sig.items():
-            f = getattr(L, name)
-            f.restype = res
-            f.argtypes = args
-        _lib = L
+        _lib = load_library(library_path)
     return _lib
 
 
@@ -153,9 +161,10 @@ def awq_quantize_pack(W: torch.Tensor, s: torch.Tensor | None, bits: int = 4,
 def awq_search_scale(W: torch.Tensor, X: torch.Tensor, s_x: torch.Tensor | None,
                      alphas: torch.Tensor | None, bits: int = 4, group: int = GROUP,
                      s_table: torch.Tensor | None = None, row_losses: bool = False,
-                     workspace=None, stream=None):
+                     workspace=None, stream=None, inv: bool = False):
     """Grid search of the per-channel scale. Returns (losses fp64 [A], best_idx int32 [1],
-    best_s fp32 [K], row_losses fp64 [A, N] or None)."""
+    best_s fp32 [K], row_losses fp64 [A, N] or None), and with ``inv=True`` a fifth item,
+    best_inv_s fp32 [K] = 1 / best_s (the GEMM's inv_s for a layer packed with best_s)."""
     _need(W, torch.float16, "W")
     _need(X, torch.float16, "X")
     _need(s_x, torch.float32, "s_x")
@@ -169,20 +178,30 @@ def awq_search_scale(W: torch.Tensor, X: torch.Tensor, s_x: torch.Tensor | None,
     best_idx = torch.empty(4, dtype=torch.int32, device=dev)
     best_s = torch.empty(K, dtype=torch.float32, device=dev)
     rl = torch.empty(A, N, dtype=torch.float64, device=dev) if row_losses else None
+    best_inv = torch.empty(K, dtype=torch.float32, device=dev) if inv else None
     ws_bytes = lib().awq_search_scale_workspace_size(M, N, K, A)
     ws = _workspace(ws_bytes, dev) if workspace is None else workspace
     _check("awq_search_scale", lib().awq_search_scale(
         _ptr(W), N, K, _ptr(X), M, _ptr(s_x), _ptr(alphas), A, bits, group, _ptr(s_table),
-        _ptr(losses), _ptr(best_idx), _ptr(best_s), _ptr(rl), _ptr(ws),
+        _ptr(losses), _ptr(best_idx), _ptr(best_s), _ptr(best_inv), _ptr(rl), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+    if inv:
+        return losses, best_idx[:1], best_s, rl, best_inv
     return losses, best_idx[:1], best_s, rl
+
+
+WEIGHTS_READY = 1   # AWQ_GEMM_WEIGHTS_READY
 
 
 def awq_gemm_w4a16(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
                    zeros: torch.Tensor, N: int, K: int, bits: int = 4, group: int = GROUP,
                    inv_s: torch.Tensor | None = None, out: torch.Tensor | None = None,
-                   workspace=None, stream=None) -> torch.Tensor:
-    """Y = X deq(W)^T (fp16 [M, N]) with the dequantization fused into the kernel."""
+                   workspace=None, stream=None, weights_ready: bool = False) -> torch.Tensor:
+    """Y = X deq(W)^T (fp16 [M, N]) with the dequantization fused into the kernel.
+
+    ``weights_ready=True`` passes AWQ_GEMM_WEIGHTS_READY: the packed weights are not written
+    by the kernel launched just before this call on the stream, so the kernel may start
+    reading them while that kernel still runs."""
     _need(X, torch.float16, "X")
     _need(scales, torch.float16, "scales")
     _need(zeros, torch.uint8, "zeros")
@@ -196,5 +215,5 @@ def awq_gemm_w4a16(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("awq_gemm_w4a16", lib().awq_gemm_w4a16(
         _ptr(X), M, _ptr(qweight), _ptr(scales), _ptr(zeros), N, K, bits, group, _ptr(inv_s),
-        _ptr(Y), _ptr(ws), ws_bytes, _stream(stream)))
+        WEIGHTS_READY if weights_ready else 0, _ptr(Y), _ptr(ws), ws_bytes, _stream(stream)))
     return Y

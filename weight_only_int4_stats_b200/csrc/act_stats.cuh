@@ -37,7 +37,10 @@ __global__ void __launch_bounds__(256) act_stats_partial_kernel(const __half* __
     for (; r + 3 * kStatsRowLanes < r1; r += 4 * kStatsRowLanes) {
       uint4 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = ldg_nc_v4(p + (r + u * kStatsRowLanes) * K);
+      for (int u = 0; u < 4; ++u)
+        v[u] = AWQ_IN_BOUNDS(r + u * kStatsRowLanes < M && col0 + 8 <= K)
+                   ? ldg_nc_v4(p + (r + u * kStatsRowLanes) * K)
+                   : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const __half2* h = reinterpret_cast<const __half2*>(&v[u]);
@@ -50,7 +53,8 @@ __global__ void __launch_bounds__(256) act_stats_partial_kernel(const __half* __
       }
     }
     for (; r < r1; r += kStatsRowLanes) {
-      uint4 v = ldg_nc_v4(p + r * K);
+      uint4 v = AWQ_IN_BOUNDS(r < M && col0 + 8 <= K) ? ldg_nc_v4(p + r * K)
+                                                       : make_uint4(0u, 0u, 0u, 0u);
       const __half2* h = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -71,7 +75,7 @@ __global__ void __launch_bounds__(256) act_stats_partial_kernel(const __half* __
     double s = 0.0;
 #pragma unroll
     for (int j = 0; j < kStatsRowLanes; ++j) s += red[j][t];
-    part[static_cast<int64_t>(blockIdx.y) * K + c] = s;
+    if (AWQ_IN_BOUNDS(blockIdx.y < gridDim.y)) part[static_cast<int64_t>(blockIdx.y) * K + c] = s;
   }
 }
 

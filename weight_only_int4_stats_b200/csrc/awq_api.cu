@@ -159,43 +159,64 @@ awq_status launch_tc_bn(const __half* Xop, int64_t M, const void* Aop, int64_t a
 }
 
 // Streaming decode GEMM (M <= 16, 4-bit), launched with programmatic dependent launch.
-// Returns AWQ_ERR_UNSUPPORTED when the shape does not suit it (X does not fit in shared
-// memory, or N is not a multiple of 16); the caller then uses the register-streaming kernel.
 constexpr int kSmemLimit = 232448;   // 227 KB per CTA on sm_100
+// Two CTAs share an SM's 228 KB when each stays within this (1 KB per CTA is reserved).
+constexpr int kCoResidentSmem = (233472 - 2 * 1024) / 2;
 
-// Whether the streaming decode kernel takes this shape: N in whole 16-row tiles and X plus
-// the weight ring within one CTA's shared memory (kNTiles = 1 for M <= 8, 2 for M <= 16).
-bool gemv_stream_fits(int64_t M, int64_t N, int64_t K) {
+static_assert(awq::kGemvWeightsReady == AWQ_GEMM_WEIGHTS_READY, "flag values must agree");
+
+struct GemvConfig {
+  int cw;       // consumer warps (8 or 16)
+  int slots;    // ring depth
+  int per_sm;   // CTAs of this grid per SM
+  int smem;     // dynamic shared memory per CTA
+  awq::G4Smem lay;
+};
+
+// The launch shape of the streaming decode kernel: 8 consumer warps, one CTA per SM and the
+// deepest ring (up to kGSMaxSlots) that leaves room for the next launch's CTA on the same SM;
+// when X is too large for that, the deepest ring within one CTA's shared memory. Returns
+// false when the shape does not suit the kernel: N not in whole 16-row tiles, or X plus a
+// two-slot ring beyond one CTA's shared memory (kNTiles = 1 for M <= 8, 2 for M <= 16).
+bool gemv_config(int64_t M, int64_t N, int64_t K, int cw, int slots_max, int per_sm,
+                 GemvConfig* out) {
   if (M < 1 || M > 16 || N % 16 != 0 || K / awq::kGroup > 65535) return false;
   if (M * K * 2 > kSmemLimit) return false;
   const int nt = M <= 8 ? 1 : 2;
-  return awq::G4Smem::make(static_cast<int>(M), K, nt).total(nt) <= kSmemLimit;
+  for (int budget : {kCoResidentSmem, kSmemLimit}) {
+    for (int slots = slots_max; slots >= 2; --slots) {
+      const awq::G4Smem l = awq::G4Smem::make(static_cast<int>(M), K, nt, slots, cw);
+      if (l.total(nt) <= budget) {
+        *out = GemvConfig{cw, slots, per_sm, l.total(nt), l};
+        return true;
+      }
+    }
+  }
+  return false;
 }
 
-template <int kNTiles, bool kOffset>
-awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweight,
-                              const __half* scales, const uint8_t* zeros, int64_t N, int64_t K,
-                              const float* inv_s, __half* y, cudaStream_t st) {
-  if (!gemv_stream_fits(M, N, K)) return AWQ_ERR_UNSUPPORTED;
-  const awq::G4Smem lay = awq::G4Smem::make(static_cast<int>(M), K, kNTiles);
-  const int smem = lay.total(kNTiles);
+bool gemv_stream_fits(int64_t M, int64_t N, int64_t K) {
+  GemvConfig c;
+  return gemv_config(M, N, K, 8, awq::kGSMaxSlots, 1, &c);
+}
+
+template <int kNTiles, bool kOffset, int kCW>
+awq_status launch_gemv_stream_cfg(const GemvConfig& cfgv, const __half* x, int64_t M,
+                                  const uint32_t* qweight, const __half* scales,
+                                  const uint8_t* zeros, int64_t N, int64_t K, const float* inv_s,
+                                  unsigned flags, __half* y, cudaStream_t st) {
   static std::atomic<bool> attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
-  auto kern = awq::gemv_stream_kernel<kNTiles, kOffset>;
+  auto kern = awq::gemv_stream_kernel<kNTiles, kOffset, kCW>;
   if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
         cudaSuccess)
       return AWQ_ERR_CUDA;
     attr_set[dev].store(true, std::memory_order_release);
   }
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, awq::kG4Threads, smem) !=
-          cudaSuccess ||
-      per_sm < 1)
-    return AWQ_ERR_CUDA;
   const int64_t tiles = N / 16;
-  const int64_t resident = static_cast<int64_t>(num_sms()) * per_sm;
+  const int64_t resident = static_cast<int64_t>(num_sms()) * cfgv.per_sm;
   const unsigned grid = static_cast<unsigned>(tiles < resident ? tiles : resident);
   CUtensorMap tw, ts, tz;
   if (!make_tmap_2d(&tw, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, 16,
@@ -207,8 +228,8 @@ awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweigh
     return AWQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(awq::kG4Threads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.blockDim = dim3((kCW + 1) * 32);
+  cfg.dynamicSmemBytes = static_cast<size_t>(cfgv.smem);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -216,32 +237,58 @@ awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweigh
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int m32 = static_cast<int>(M);
-  if (cudaLaunchKernelEx(&cfg, kern, tw, ts, tz, qweight, x, m32, N, K, inv_s, y, lay) !=
-      cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kern, tw, ts, tz, qweight, x, m32, N, K, inv_s, y, cfgv.lay,
+                         flags) != cudaSuccess)
     return AWQ_ERR_CUDA;
   return launch_status();
+}
+
+// Returns AWQ_ERR_UNSUPPORTED when the shape does not suit the streaming kernel; the caller
+// then uses the register-streaming kernel (M <= 8) or the tensor-core path.
+awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweight,
+                              const __half* scales, const uint8_t* zeros, int64_t N, int64_t K,
+                              const float* inv_s, unsigned flags, __half* y, cudaStream_t st) {
+  GemvConfig c;
+  if (!gemv_config(M, N, K, 8, awq::kGSMaxSlots, 1, &c)) return AWQ_ERR_UNSUPPORTED;
+  if (M == 1)
+    return launch_gemv_stream_cfg<1, true, 8>(c, x, M, qweight, scales, zeros, N, K, inv_s,
+                                              flags, y, st);
+  if (M <= 8)
+    return launch_gemv_stream_cfg<1, false, 8>(c, x, M, qweight, scales, zeros, N, K, inv_s,
+                                               flags, y, st);
+  return launch_gemv_stream_cfg<2, false, 8>(c, x, M, qweight, scales, zeros, N, K, inv_s,
+                                             flags, y, st);
 }
 
 int tc_bn_for(int64_t M) { return M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
 // Split-K for the tensor-core GEMM when the output has too few 128 x BN tiles to occupy the
-// GPU (batched decode, small prefill): fill one wave of resident CTAs, keep at least two
-// groups per slice, and keep the fp32 partial traffic (8 bytes per output and slice) within
-// about the packed weight bytes.
+// GPU (batched decode, small prefill). The persistent kernel runs one CTA per SM and hands
+// out (tile, K slice) units round-robin, so the busiest SM does ceil(tiles * s / sms) units
+// of K / s each: pick the split s that minimises that, i.e. ceil(tiles * s / sms) / s (a
+// later s must win by more than 2% per extra slice, since each slice adds 8 bytes of fp32
+// partial sums per output), with at least two 128-wide groups per slice and the partial
+// traffic within about the packed weight bytes.
 int splitk_for(int64_t M, int64_t N, int64_t K) {
   const int64_t bn = tc_bn_for(M);
   const int64_t tiles = ((N + awq::kTcBM - 1) / awq::kTcBM) * ((M + bn - 1) / bn);
   const int64_t sms = num_sms();
-  // the persistent kernel runs one CTA per SM: fill the SMs once, with about one work unit
-  // per SM (more would only queue behind each other)
   if (tiles >= sms) return 1;
-  int64_t s = sms / tiles;
-  const int64_t by_groups = (K / awq::kGroup) / 2;
+  int64_t s_max = (K / awq::kGroup) / 2;
   const int64_t by_traffic = K / (8 * M);
-  if (s > by_groups) s = by_groups;
-  if (s > by_traffic) s = by_traffic;
-  if (s > 16) s = 16;
-  return s < 2 ? 1 : static_cast<int>(s);
+  if (s_max > by_traffic) s_max = by_traffic;
+  if (s_max > 16) s_max = 16;
+  int best = 1;
+  double best_cost = 1.0;
+  for (int64_t s = 2; s <= s_max; ++s) {
+    const double cost =
+        static_cast<double>((tiles * s + sms - 1) / sms) / static_cast<double>(s);
+    if (cost * (1.0 + 0.02 * static_cast<double>(s - best)) < best_cost) {
+      best = static_cast<int>(s);
+      best_cost = cost;
+    }
+  }
+  return best;
 }
 
 bool bad_dim(int64_t v) { return v < 0 || v > kMaxDim; }
@@ -258,11 +305,12 @@ const char* awq_status_string(awq_status status) {
     case AWQ_ERR_WORKSPACE: return "AWQ_ERR_WORKSPACE";
     case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA";
     case AWQ_ERR_TIMEOUT: return "AWQ_ERR_TIMEOUT";
+    case AWQ_ERR_BOUNDS: return "AWQ_ERR_BOUNDS";
   }
   return "AWQ_ERR_UNKNOWN";
 }
 
-int awq_abi_version(void) { return 1; }
+int awq_abi_version(void) { return 2; }
 
 awq_status awq_check_error(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -272,8 +320,21 @@ awq_status awq_check_error(void* stream) {
     return AWQ_ERR_CUDA;
   if (word != 0 && cudaMemcpyToSymbol(awq::g_status_word, &zero, sizeof(zero)) != cudaSuccess)
     return AWQ_ERR_CUDA;
+  if (word & awq::kDevErrBounds) return AWQ_ERR_BOUNDS;
   if (word & awq::kDevErrTimeout) return AWQ_ERR_TIMEOUT;
   return AWQ_OK;
+}
+
+awq_status awq_selftest_bounds(int* buf, void* stream) {
+#ifdef AWQ_DEBUG_BOUNDS
+  if (buf == nullptr || (reinterpret_cast<uintptr_t>(buf) & 15u) != 0) return AWQ_ERR_INVALID_ARG;
+  awq::bounds_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(buf, 4);
+  return launch_status();
+#else
+  (void)buf;
+  (void)stream;
+  return AWQ_ERR_UNSUPPORTED;   // the release build has no bounds checks
+#endif
 }
 
 awq_status awq_selftest_timeout(int* waited_out, void* stream) {
@@ -399,18 +460,29 @@ awq_status awq_quantize_pack(const awq_f16* W, int64_t N, int64_t K, const float
 
 // ------------------------------------------------------------------ search
 namespace {
+// The error operand E is built and reduced for a chunk of grid points at a time, so the
+// workspace stays bounded whatever the layer: at most this many bytes of E per chunk (at
+// least one grid point per chunk).
+constexpr size_t kSearchChunkBytes = size_t{1} << 30;
+
 struct SearchWs {
+  int chunk;   // grid points per chunk
   size_t table, inv, err, part, rows, total;
 };
 SearchWs search_ws_layout(int64_t M, int64_t N, int64_t K, int n_alpha) {
   const int64_t N_pad = round_up(N, awq::kTcBM);
   const int64_t m_tiles = (M + tc_bn_for(M) - 1) / tc_bn_for(M);
+  const size_t per_point = static_cast<size_t>(N_pad) * K * sizeof(__half);
+  int64_t chunk = static_cast<int64_t>(kSearchChunkBytes / per_point);
+  if (chunk < 1) chunk = 1;
+  if (chunk > n_alpha) chunk = n_alpha;
   SearchWs w;
+  w.chunk = static_cast<int>(chunk);
   w.table = 0;
   w.inv = align256(static_cast<size_t>(n_alpha) * K * sizeof(float));
   w.err = w.inv + align256(static_cast<size_t>(n_alpha) * K * sizeof(float));
-  w.part = w.err + align256(static_cast<size_t>(n_alpha) * N_pad * K * sizeof(__half));
-  w.rows = w.part + align256(static_cast<size_t>(n_alpha) * N_pad * m_tiles * sizeof(double));
+  w.part = w.err + align256(static_cast<size_t>(chunk) * per_point);
+  w.rows = w.part + align256(static_cast<size_t>(chunk) * N_pad * m_tiles * sizeof(double));
   w.total = w.rows + align256(static_cast<size_t>(n_alpha) * N * sizeof(double));
   return w;
 }
@@ -424,8 +496,9 @@ size_t awq_search_scale_workspace_size(int64_t M, int64_t N, int64_t K, int n_al
 awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f16* X,
                             int64_t M, const float* s_x, const float* alphas, int n_alpha,
                             int bits, int group, const float* s_table, double* losses,
-                            int32_t* best_idx, float* best_s, double* row_losses,
-                            void* workspace, size_t ws_bytes, void* stream) {
+                            int32_t* best_idx, float* best_s, float* best_inv_s,
+                            double* row_losses, void* workspace, size_t ws_bytes,
+                            void* stream) {
   if (bad_dim(N) || bad_dim(K) || bad_dim(M) || N == 0 || K == 0 || M == 0)
     return AWQ_ERR_INVALID_ARG;
   if (group != awq::kGroup || K % awq::kGroup != 0) return AWQ_ERR_INVALID_ARG;
@@ -435,12 +508,13 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
   if (!s_table && (!s_x || !alphas)) return AWQ_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(X) || !aligned16(losses) || !aligned16(best_idx) ||
       !aligned16(best_s) || (s_x && !aligned16(s_x)) || (alphas && !aligned16(alphas)) ||
-      (s_table && !aligned16(s_table)) || (row_losses && !aligned16(row_losses)))
+      (s_table && !aligned16(s_table)) || (row_losses && !aligned16(row_losses)) ||
+      (best_inv_s && !aligned16(best_inv_s)))
     return AWQ_ERR_INVALID_ARG;
   const int64_t N_pad = round_up(N, awq::kTcBM);
-  if (n_alpha * N_pad / awq::kTcBM > 65535 || K / awq::kGroup > 65535)
-    return AWQ_ERR_INVALID_ARG;
+  if (N_pad / awq::kTcBM > 65535 || K / awq::kGroup > 65535) return AWQ_ERR_INVALID_ARG;
   const SearchWs lay = search_ws_layout(M, N, K, n_alpha);
+  if (static_cast<int64_t>(lay.chunk) * N_pad / awq::kTcBM > 65535) return AWQ_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < lay.total || !aligned16(workspace)) return AWQ_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -464,41 +538,47 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
     awq::inv_table_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(S, total, inv);
     if ((s = launch_status()) != AWQ_OK) return s;
   }
-  {
-    dim3 g(static_cast<unsigned>(N_pad / awq::kQuantRowsPerCta),
-           static_cast<unsigned>(K / awq::kGroup), static_cast<unsigned>(n_alpha));
-    const __half* w = reinterpret_cast<const __half*>(W);
-    if (bits == 4)
-      awq::search_build_error_kernel<4><<<g, 256, 0, st>>>(w, N, K, N_pad, S, inv, E);
-    else
-      awq::search_build_error_kernel<3><<<g, 256, 0, st>>>(w, N, K, N_pad, S, inv, E);
-    if ((s = launch_status()) != AWQ_OK) return s;
-  }
-  {
-    awq::TcArgs args{};
-    args.M = M;
-    args.N = N;
-    args.N_pad = N_pad;
-    args.K = K;
-    args.row_part = part;
-    args.m_tiles = m_tiles;
-    args.k_splits = 1;
-    s = launch_tc_bn<ASrc::kFp16, Epi::kRowSumSq>(reinterpret_cast<const __half*>(X), M, E,
-                                                  n_alpha * N_pad, args, st);
-    if (s != AWQ_OK) return s;
-  }
   double* rl = row_losses != nullptr ? row_losses : reinterpret_cast<double*>(ws + lay.rows);
-  {
-    const int64_t n = static_cast<int64_t>(n_alpha) * N;
-    awq::search_row_loss_kernel<<<static_cast<unsigned>((n + awq::kReduceThreads - 1) /
-                                                        awq::kReduceThreads),
-                                  awq::kReduceThreads, 0, st>>>(part, N, N_pad, n_alpha, m_tiles, rl);
-    if ((s = launch_status()) != AWQ_OK) return s;
+  const __half* w = reinterpret_cast<const __half*>(W);
+  for (int a0 = 0; a0 < n_alpha; a0 += lay.chunk) {
+    const int na = n_alpha - a0 < lay.chunk ? n_alpha - a0 : lay.chunk;
+    const float* Sa = S + static_cast<int64_t>(a0) * K;
+    const float* Ia = inv + static_cast<int64_t>(a0) * K;
+    {
+      dim3 g(static_cast<unsigned>(N_pad / awq::kQuantRowsPerCta),
+             static_cast<unsigned>(K / awq::kGroup), static_cast<unsigned>(na));
+      if (bits == 4)
+        awq::search_build_error_kernel<4><<<g, 256, 0, st>>>(w, N, K, N_pad, Sa, Ia, E);
+      else
+        awq::search_build_error_kernel<3><<<g, 256, 0, st>>>(w, N, K, N_pad, Sa, Ia, E);
+      if ((s = launch_status()) != AWQ_OK) return s;
+    }
+    {
+      awq::TcArgs args{};
+      args.M = M;
+      args.N = N;
+      args.N_pad = N_pad;
+      args.K = K;
+      args.row_part = part;
+      args.m_tiles = m_tiles;
+      args.k_splits = 1;
+      s = launch_tc_bn<ASrc::kFp16, Epi::kRowSumSq>(reinterpret_cast<const __half*>(X), M, E,
+                                                    na * N_pad, args, st);
+      if (s != AWQ_OK) return s;
+    }
+    {
+      const int64_t n = static_cast<int64_t>(na) * N;
+      awq::search_row_loss_kernel<<<static_cast<unsigned>((n + awq::kReduceThreads - 1) /
+                                                          awq::kReduceThreads),
+                                    awq::kReduceThreads, 0, st>>>(part, N, N_pad, na, m_tiles,
+                                                                  rl + static_cast<int64_t>(a0) * N);
+      if ((s = launch_status()) != AWQ_OK) return s;
+    }
   }
   awq::search_reduce_kernel<<<n_alpha, awq::kReduceThreads, 0, st>>>(rl, N, losses);
   if ((s = launch_status()) != AWQ_OK) return s;
   awq::search_pick_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(
-      losses, n_alpha, S, K, best_idx, best_s);
+      losses, n_alpha, S, inv, K, best_idx, best_s, best_inv_s);
   return launch_status();
 }
 
@@ -509,15 +589,13 @@ size_t awq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits) {
   // takes the tensor-core path below
   if (M <= 16 && bits == 4 && (M <= 8 || gemv_stream_fits(M, N, K))) return 0;
   const int splits = splitk_for(M, N, K);
-  size_t bytes = align256(static_cast<size_t>(M) * K * sizeof(__half));   // x * inv_s
-  if (splits > 1) bytes += align256(static_cast<size_t>(splits) * M * N * sizeof(float));
-  return bytes;
+  return splits > 1 ? align256(static_cast<size_t>(splits) * M * N * sizeof(float)) : 0;
 }
 
 awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
                           const awq_f16* scales, const uint8_t* zeros, int64_t N, int64_t K,
-                          int bits, int group, const float* inv_s, awq_f16* Y, void* workspace,
-                          size_t ws_bytes, void* stream) {
+                          int bits, int group, const float* inv_s, unsigned flags, awq_f16* Y,
+                          void* workspace, size_t ws_bytes, void* stream) {
   if (bad_dim(M) || bad_dim(N) || bad_dim(K) || K == 0) return AWQ_ERR_INVALID_ARG;
   if (group != awq::kGroup || K % awq::kGroup != 0) return AWQ_ERR_INVALID_ARG;
   if (bits != 4 && bits != 3) return AWQ_ERR_INVALID_ARG;
@@ -526,16 +604,14 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
   if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
       !aligned16(Y) || (inv_s && !aligned16(inv_s)))
     return AWQ_ERR_INVALID_ARG;
+  if ((flags & ~static_cast<unsigned>(AWQ_GEMM_WEIGHTS_READY)) != 0) return AWQ_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const __half* x = reinterpret_cast<const __half*>(X);
   const __half* sc = reinterpret_cast<const __half*>(scales);
   __half* y = reinterpret_cast<__half*>(Y);
 
   if (M <= 16 && bits == 4) {
-    awq_status r =
-        M == 1  ? launch_gemv_stream<1, true>(x, M, qweight, sc, zeros, N, K, inv_s, y, st)
-        : M <= 8 ? launch_gemv_stream<1, false>(x, M, qweight, sc, zeros, N, K, inv_s, y, st)
-                 : launch_gemv_stream<2, false>(x, M, qweight, sc, zeros, N, K, inv_s, y, st);
+    awq_status r = launch_gemv_stream(x, M, qweight, sc, zeros, N, K, inv_s, flags, y, st);
     if (r != AWQ_ERR_UNSUPPORTED) return r;
     // the streaming kernel cannot hold X (or N % 16 != 0): register streaming for M <= 8,
     // the tensor-core path below for 8 < M <= 16
@@ -547,26 +623,12 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
     }
   }
   if ((N + awq::kTcBM - 1) / awq::kTcBM > 65535) return AWQ_ERR_INVALID_ARG;
-  const __half* xop = x;
   const int splits = splitk_for(M, N, K);
-  const size_t xs_bytes = align256(static_cast<size_t>(M) * K * sizeof(__half));
   const size_t part_bytes =
       splits > 1 ? align256(static_cast<size_t>(splits) * M * N * sizeof(float)) : 0;
-  const size_t need = (inv_s != nullptr ? xs_bytes : 0) + part_bytes;
-  if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
+  if (part_bytes > 0 && (!workspace || ws_bytes < part_bytes || !aligned16(workspace)))
     return AWQ_ERR_WORKSPACE;
-  float* partial = splits > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                                        (inv_s != nullptr ? xs_bytes : 0))
-                              : nullptr;
-  if (inv_s != nullptr) {
-    __half* xs = static_cast<__half*>(workspace);
-    const int64_t n8 = M * K / 8;
-    awq::prescale_x_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, st>>>(x, inv_s, M,
-                                                                                   K, xs);
-    awq_status s = launch_status();
-    if (s != AWQ_OK) return s;
-    xop = xs;
-  }
+  float* partial = splits > 1 ? static_cast<float*>(workspace) : nullptr;
   awq::TcArgs args{};
   args.M = M;
   args.N = N;
@@ -578,9 +640,10 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
   args.m_tiles = static_cast<int>((M + tc_bn_for(M) - 1) / tc_bn_for(M));
   args.k_splits = splits;
   args.partial = partial;
+  args.inv_s = inv_s;   // folded into the dequantized weights by the builders
   awq_status r =
-      bits == 3 ? launch_tc_bn<ASrc::kPacked3, Epi::kStoreY>(xop, M, qweight, N, args, st)
-                : launch_tc_bn<ASrc::kPacked4, Epi::kStoreY>(xop, M, qweight, N, args, st);
+      bits == 3 ? launch_tc_bn<ASrc::kPacked3, Epi::kStoreY>(x, M, qweight, N, args, st)
+                : launch_tc_bn<ASrc::kPacked4, Epi::kStoreY>(x, M, qweight, N, args, st);
   if (r != AWQ_OK || splits == 1) return r;
   const int64_t MN = M * N;
   awq::splitk_reduce_kernel<<<static_cast<unsigned>((MN / 4 + 1 + 255) / 256), 256, 0, st>>>(

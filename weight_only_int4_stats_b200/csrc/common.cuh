@@ -31,6 +31,20 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 
 __device__ __forceinline__ void flag_error(unsigned bits) { atomicOr(&g_status_word, bits); }
 
+// Index checks of the debug build (compiled with AWQ_DEBUG_BOUNDS): AWQ_IN_BOUNDS(cond) is
+// false, and records kDevErrBounds in the status word, when an index the kernel is about to
+// use falls outside the extent the call's shapes give; the kernel then skips that access. In
+// the release build it is the constant true and compiles away.
+#ifdef AWQ_DEBUG_BOUNDS
+__device__ __forceinline__ bool bounds_ok(bool cond) {
+  if (!cond) flag_error(kDevErrBounds);
+  return cond;
+}
+#define AWQ_IN_BOUNDS(cond) (::awq::bounds_ok(cond))
+#else
+#define AWQ_IN_BOUNDS(cond) (true)
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -115,6 +129,16 @@ __global__ void timeout_selftest_kernel(unsigned long long limit_ns, int* waited
     *waited_out = ok ? 0 : 1;
   }
 }
+
+#ifdef AWQ_DEBUG_BOUNDS
+// Self-test of the debug build's bounds checks: one thread walks one index past a buffer of
+// n ints; the check stops the last store and records the violation.
+__global__ void bounds_selftest_kernel(int* buf, int n) {
+  if (threadIdx.x == 0)
+    for (int i = 0; i <= n; ++i)
+      if (AWQ_IN_BOUNDS(i < n)) buf[i] = i;
+}
+#endif
 
 // ----------------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

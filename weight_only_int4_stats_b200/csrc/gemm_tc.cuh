@@ -103,6 +103,7 @@ struct TcArgs {
   float* partial;       // [k_splits, M, N] fp32 partial sums (split-K store epilogue)
   int sz_tma;           // packed source: scales and zeros arrive by TMA with the packed group
                         // (needs N % 16 == 0); else the builders load them from global memory
+  const float* inv_s;   // packed source: NULL, or [K] factors folded into the weights
 };
 
 // Grouped tile order: consecutive work units sweep the token tiles of a group of
@@ -138,9 +139,11 @@ __device__ __forceinline__ TcUnit unit_of(int64_t u, const TcArgs& a) {
   return t;
 }
 
-// Dequantize one 4-bit packed word (8 consecutive k) to four fp16 pairs (q - z) * sc.
+// Dequantize one 4-bit packed word (8 consecutive k) to four fp16 pairs (q - z) * c, with
+// one scale pair per k pair: (k0,k1) by c.x, (k2,k3) by c.y, (k4,k5) by c.z, (k6,k7) by c.w
+// (all four the group's scale, or the scale times the per-channel inv_s).
 __device__ __forceinline__ uint4 dequant_word_scaled(uint32_t w, __half2 bias_lo,
-                                                     __half2 bias_hi, __half2 sc2) {
+                                                     __half2 bias_hi, uint4 c) {
   const __half2 sixteenth = __float2half2_rn(0.0625f);
   const uint32_t w8 = w >> 8;
   const uint32_t v0 = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
@@ -148,11 +151,28 @@ __device__ __forceinline__ uint4 dequant_word_scaled(uint32_t w, __half2 bias_lo
   const uint32_t v2 = lop3_and_or(w8, 0x000F000Fu, 0x64006400u);
   const uint32_t v3 = lop3_and_or(w8, 0x00F000F0u, 0x64006400u);
   uint4 o;
-  o.x = h2_as_u32(__hmul2(__hsub2(u32_as_h2(v0), bias_lo), sc2));
-  o.y = h2_as_u32(__hmul2(__hfma2(u32_as_h2(v1), sixteenth, bias_hi), sc2));
-  o.z = h2_as_u32(__hmul2(__hsub2(u32_as_h2(v2), bias_lo), sc2));
-  o.w = h2_as_u32(__hmul2(__hfma2(u32_as_h2(v3), sixteenth, bias_hi), sc2));
+  o.x = h2_as_u32(__hmul2(__hsub2(u32_as_h2(v0), bias_lo), u32_as_h2(c.x)));
+  o.y = h2_as_u32(__hmul2(__hfma2(u32_as_h2(v1), sixteenth, bias_hi), u32_as_h2(c.y)));
+  o.z = h2_as_u32(__hmul2(__hsub2(u32_as_h2(v2), bias_lo), u32_as_h2(c.z)));
+  o.w = h2_as_u32(__hmul2(__hfma2(u32_as_h2(v3), sixteenth, bias_hi), u32_as_h2(c.w)));
   return o;
+}
+
+// The four scale pairs of 8 consecutive k starting at k0: fp16(sc * inv_s[k]) pairs, or sc
+// broadcast when inv_s is NULL. Folding inv_s into the weights computes
+// sum_k x[k] * (inv_s[k] * deq[k]) = sum_k (x[k] * inv_s[k]) * deq[k].
+__device__ __forceinline__ uint4 pair_scales(float sc, __half2 sc2, const float* inv_s,
+                                             int64_t k0) {
+  if (inv_s == nullptr) {
+    const uint32_t s = h2_as_u32(sc2);
+    return make_uint4(s, s, s, s);
+  }
+  const float4 a = *reinterpret_cast<const float4*>(inv_s + k0);
+  const float4 b = *reinterpret_cast<const float4*>(inv_s + k0 + 4);
+  return make_uint4(h2_as_u32(__floats2half2_rn(sc * a.x, sc * a.y)),
+                    h2_as_u32(__floats2half2_rn(sc * a.z, sc * a.w)),
+                    h2_as_u32(__floats2half2_rn(sc * b.x, sc * b.y)),
+                    h2_as_u32(__floats2half2_rn(sc * b.z, sc * b.w)));
 }
 
 // 3-bit: the fp16 pair (q - z) * sc for k-offsets (2e, 2e+1) of chunk i (k = 8i..8i+7) of a
@@ -161,7 +181,8 @@ __device__ __forceinline__ uint4 dequant_word_scaled(uint32_t w, __half2 bias_lo
 // 16-bit half by a single shift whose direction is fixed at compile time).
 template <int kI, int kE>
 __device__ __forceinline__ uint32_t dequant3_pair(uint32_t w0, uint32_t w1, uint32_t w2,
-                                                  __half2 bias_lo, __half2 sc2) {
+                                                  __half2 bias_lo, uint32_t sc2u) {
+  const __half2 sc2 = u32_as_h2(sc2u);
   constexpr int pp = 4 * (kI & 1) + kE;     // 2-bit field of the pair inside its low word
   constexpr int hb = 4 * kI + kE;           // bit of the pair inside the bit-2 word
   const uint32_t wlo = (kI < 2) ? w0 : w1;
@@ -240,9 +261,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   // Programmatic dependent launch: the setup above may overlap the previous kernel on the
   // stream; every thread waits for that kernel's completion (and memory) before its first
-  // global access, and lets the next kernel launch early.
-  pdl_launch_dependents();
+  // global access, and only then lets the next kernel launch (so a kernel that starts early
+  // behind this one overlaps this kernel alone, never an earlier one).
   pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == kTcXWarp) {
     // ------------------------------------------------------------------ TMA producer
@@ -324,7 +346,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           __half sv = __float2half(0.0f);
           if (!args.sz_tma) {   // ragged N: this row's zero point and scale from global
             const int64_t g = kb >> 1;
-            if (n < N) {
+            if (n < N && AWQ_IN_BOUNDS(g < args.K / kGroup)) {
               z = args.zeros[g * N + n];
               sv = args.scales[g * N + n];
             }
@@ -338,6 +360,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           ok = __all_sync(0xffffffffu, got);   // keep the warp converged for .aligned ops
           if (!ok) break;
           const int gi = (i >> 1) % L::kPG;          // group inside the slot
+          if (!AWQ_IN_BOUNDS(ps < P && s < S && s1 < S && kb + 2 <= 2 * (args.K / kGroup))) {
+            ok = false;
+            break;
+          }
           if (args.sz_tma) {   // rows past N were filled with zeros by the TMA unit
             const uint8_t* sz = smem + L::kSZOff + ps * L::kSZBytes;
             sv = reinterpret_cast<const __half*>(sz)[gi * kTcBM + r];
@@ -346,6 +372,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const __half2 lo = u32_as_h2((0x6400u | z) * 0x00010001u);
           const __half2 hi = u32_as_h2((0xD400u | (z << 4)) * 0x00010001u);
           const __half2 sc = __half2half2(sv);
+          const float scf = __half2float(sv);
           const uint8_t* prow = smem + L::kPOff + ps * L::kPBytes + r * L::kPRowBytes;
 #pragma unroll
           for (int e = 0; e < 2; ++e) {             // stage i + e of the group
@@ -356,19 +383,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                const uint4 o = dequant_word_scaled(words[q], lo, hi, sc);
+                const int64_t k0 = static_cast<int64_t>(kb + e) * kTcBK + 32 * h + 8 * q;
+                const uint4 c4 = pair_scales(scf, sc, args.inv_s, k0);
+                const uint4 o = dequant_word_scaled(words[q], lo, hi, c4);
                 *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + q)) = o;
               }
             } else {
               const uint32_t* pw =
                   reinterpret_cast<const uint32_t*>(prow + gi * 48 + 12 * (2 * e + h));
               const uint32_t w0 = pw[0], w1 = pw[1], w2 = pw[2];
-              uint4 o;
-#define AWQ_DQ3_CHUNK(I)                                                   \
-  o.x = dequant3_pair<I, 0>(w0, w1, w2, lo, sc);                          \
-  o.y = dequant3_pair<I, 1>(w0, w1, w2, lo, sc);                          \
-  o.z = dequant3_pair<I, 2>(w0, w1, w2, lo, sc);                          \
-  o.w = dequant3_pair<I, 3>(w0, w1, w2, lo, sc);                          \
+              uint4 o, c4;
+#define AWQ_DQ3_CHUNK(I)                                                                    \
+  c4 = pair_scales(scf, sc, args.inv_s,                                                    \
+                   static_cast<int64_t>(kb + e) * kTcBK + 32 * h + 8 * (I));               \
+  o.x = dequant3_pair<I, 0>(w0, w1, w2, lo, c4.x);                                         \
+  o.y = dequant3_pair<I, 1>(w0, w1, w2, lo, c4.y);                                         \
+  o.z = dequant3_pair<I, 2>(w0, w1, w2, lo, c4.z);                                         \
+  o.w = dequant3_pair<I, 3>(w0, w1, w2, lo, c4.w);                                         \
   *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + I)) = o;
               AWQ_DQ3_CHUNK(0)
               AWQ_DQ3_CHUNK(1)
@@ -407,6 +438,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int64_t arow = static_cast<int64_t>(t.row_tile) * kTcBM + row;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * wq) << 16) +
                              static_cast<uint32_t>(buf * BN);
+      const bool unit_ok = AWQ_IN_BOUNDS(t.row_tile < args.row_tiles && t.m_tile < args.m_tiles &&
+                                         t.ksplit < args.k_splits &&
+                                         (buf + 1) * BN <= static_cast<int>(L::kTmemCols));
       double sumsq = 0.0;
 #pragma unroll 1
       for (int col = 0; col < BN; col += 16) {
@@ -414,7 +448,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_ld_32x32b_x16(taddr + col, v);
         tmem_ld_wait();
         if (kEpi == Epi::kStoreY) {
-          if (arow < args.N) {
+          if (arow < args.N && unit_ok) {
             if (args.k_splits == 1) {
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
@@ -440,7 +474,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           sumsq += static_cast<double>(part);
         }
       }
-      if (kEpi == Epi::kRowSumSq)
+      if (kEpi == Epi::kRowSumSq && unit_ok && AWQ_IN_BOUNDS(arow < args.rows_total))
         args.row_part[static_cast<int64_t>(t.m_tile) * args.rows_total + arow] = sumsq;
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);            // the MMA may overwrite this accumulator
@@ -492,6 +526,7 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int k_sp
   if ((MN & 3) == 0) {   // every slice's start is 16-byte aligned
     float4 acc = *reinterpret_cast<const float4*>(partial + i);
     for (int s = 1; s < k_splits; ++s) {
+      if (!AWQ_IN_BOUNDS(i + 4 <= MN)) break;
       const float4 v = *reinterpret_cast<const float4*>(partial + static_cast<int64_t>(s) * MN + i);
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }

@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_w4a16_kernel(
   uint8_t za[kGemvPrefetch], zb[kGemvPrefetch];
   __half sa[kGemvPrefetch], sb[kGemvPrefetch];
   auto issue = [&](int slot, int64_t g) {
-    if (g < G) {
+    if (g < G && AWQ_IN_BOUNDS(g * 16 + c * 4 + 4 <= wpr)) {
       const int64_t wo = g * 16 + c * 4;
       wa[slot] = okA ? ldg_nc_v4(qweight + nA * wpr + wo) : make_uint4(0u, 0u, 0u, 0u);
       wb[slot] = okB ? ldg_nc_v4(qweight + nB * wpr + wo) : make_uint4(0u, 0u, 0u, 0u);
@@ -199,23 +199,28 @@ namespace awq {
 // Streaming decode GEMM (the decode path for M <= 16 when X fits in shared memory; an
 // 8 < M <= 16 call whose X does not fit takes the tensor-core GEMM instead).
 //
-// Persistent: the grid is sized to the resident capacity and CTA b owns the contiguous
-// range of whole 16-row tiles [b*T/P, (b+1)*T/P), so no output is split across CTAs and the
-// result does not depend on the grid. One producer thread walks the CTA's (tile, 2048-k
-// chunk) units and streams each unit's packed weights ([16 rows, 256 words] = 16 KB), fp16
-// scales and uint8 zeros ([16 groups, 16 rows]) with TMA into a 4-slot shared-memory ring.
+// Persistent: the grid is one CTA per SM (as many as there are 16-row tiles, at most) and
+// CTA b owns the contiguous range of whole 16-row tiles [b*T/P, (b+1)*T/P), so no output is
+// split across CTAs and the result does not depend on the grid. One producer thread walks
+// the CTA's (tile, 2048-k chunk) units and streams each unit's packed weights
+// ([16 rows, 256 words] = 16 KB), fp16 scales and uint8 zeros ([16 groups, 16 rows]) with
+// TMA into a shared-memory ring of up to kGSMaxSlots slots.
 //
-// Programmatic dependent launch: the kernel may start while the previous kernel on the
-// stream is still running. Before griddepcontrol.wait the producer only issues L2 bulk
-// prefetches of the CTA's weight rows (coherent with any write of that kernel, so even a
-// quantize-and-pack just before it is safe); every shared-memory load comes after the wait.
-// X ([M, K], small at decode) is then bulk-copied into shared memory once per CTA.
+// Back-to-back launches overlap (programmatic dependent launch). A CTA needs at most half of
+// an SM's shared memory, so the next GEMM's CTAs become resident beside this one's as soon as
+// every CTA of this grid has passed griddepcontrol.wait (the point where the launch of the
+// next grid is allowed). Before its own griddepcontrol.wait, a CTA touches no output and no
+// activation: it issues L2 prefetches of its weight rows (coherent with writes of the
+// preceding kernel, so always safe) and, when the caller states that the weights are not
+// written by the kernel launched just before (kGemvWeightsReady), TMA-loads the first ring
+// slots so that this GEMM's weights stream while the preceding kernel still runs. X
+// ([M, K], small at decode) is bulk-copied into shared memory after the wait.
 //
-// Eight consumer warps each take two 128-wide groups of every unit (two independent MMA
-// chains) with register-only dequantization feeding mma.sync m16n8k16 (weights as the
-// 16-row A operand, activations as the 8-column B operand). A warp copies its packed
-// words, scales and zero points of the unit to registers and releases the ring slot
-// before the arithmetic, so the producer can refill it at once. Two dequantization forms:
+// kCW consumer warps each take 16 / kCW of the unit's sixteen 128-wide groups, with
+// register-only dequantization feeding mma.sync m16n8k16 (weights as the 16-row A operand,
+// activations as the 8-column B operand). A warp copies its packed words, scales and zero
+// points of the unit to registers and releases the ring slot before the arithmetic, so the
+// producer can refill it at once. Two dequantization forms:
 //  * M = 1 (kOffset): a mask-and-or with 0x6400 turns the nibble pair (k0, k1) of a word
 //    into the exact fp16 values (1024 + q0, 1024 + q1) and the pair (k2, k3), stored 4 bits
 //    higher, into (1024 + 16 q2, 1024 + 16 q3) (the same after a shift by 8 for k4..k7);
@@ -223,35 +228,39 @@ namespace awq {
 //    16 (exact in fp16), so per group the MMA returns sum_k x_k q_k + C1 with
 //    C1 = 1024 * sum_k xs_k; with C2 = sum_k x_k the group adds s * (mma - C1 - z C2).
 //    The staging and C1, C2 are one pass over X per CTA. Five integer operations per
-//    packed word; the fp32
-//    cancellation of the 1024 offset keeps about 13 significant bits of each group sum.
+//    packed word; the fp32 cancellation of the 1024 offset keeps about 13 significant bits
+//    of each group sum.
 //  * M > 1: one fp16 subtract (or multiply-add) per pair leaves the exact q - z first.
-// Per-tile sums of the eight warps are added in a fixed order and stored as fp16.
+// Each group's eight MMAs run as four independent accumulator chains. At the end of a tile
+// the consumer warps' partial sums are added in a fixed warp order and stored as fp16.
 // ---------------------------------------------------------------------------------------
-constexpr int kG4Warps = 8;                        // consumer warps
-constexpr int kG4Threads = (kG4Warps + 1) * 32;    // + one producer warp
-constexpr int kG4Groups = 2 * kG4Warps;            // groups per unit
+constexpr int kG4Groups = 16;                      // groups per unit
 constexpr int kG4KC = kG4Groups * kGroup;          // k per unit (2048)
 constexpr int kG4WBytes = kGemvRows * (kG4KC / 2);             // 16384
 constexpr int kG4SBytes = kG4Groups * kGemvRows * 2;           // 512
 constexpr int kG4ZBytes = kG4Groups * kGemvRows;               // 256
 constexpr int kG4SlotBytes = kG4WBytes + kG4SBytes + kG4ZBytes; // 17152 (multiple of 128)
-constexpr int kG4Slots = 4;
+constexpr int kGSMaxSlots = 6;
+
+// Flag bits of the decode launch (awq_gemm_w4a16's flags).
+constexpr unsigned kGemvWeightsReady = 1u;
 
 struct G4Smem {
   int x_bytes;   // M * K * 2, rounded up to 128
   int c_bytes;   // C1/C2 per (group, token)
+  int slots;     // ring depth
+  int cw;        // consumer warps
   __host__ __device__ int c_off() const { return x_bytes; }
   __host__ __device__ int slot_off() const { return x_bytes + c_bytes; }
-  __host__ __device__ int bar_off() const { return slot_off() + kG4Slots * kG4SlotBytes; }
-  __host__ __device__ int red_off() const { return bar_off() + (2 * kG4Slots + 2) * 8; }
-  __host__ __device__ int total(int n_tiles) const {
-    return red_off() + kG4Warps * n_tiles * 4 * 32 * 4;
-  }
-  __host__ __device__ static G4Smem make(int M, int64_t K, int n_tiles) {
+  __host__ __device__ int bar_off() const { return slot_off() + slots * kG4SlotBytes; }
+  __host__ __device__ int red_off() const { return bar_off() + (2 * kGSMaxSlots + 2) * 8; }
+  __host__ __device__ int total(int n_tiles) const { return red_off() + cw * n_tiles * 4 * 32 * 4; }
+  __host__ __device__ static G4Smem make(int M, int64_t K, int n_tiles, int slots, int cw) {
     G4Smem l;
     l.x_bytes = static_cast<int>((static_cast<int64_t>(M) * K * 2 + 127) / 128 * 128);
     l.c_bytes = static_cast<int>(((K / kGroup) * 8 * n_tiles * 2 * 4 + 127) / 128 * 128);
+    l.slots = slots;
+    l.cw = cw;
     return l;
   }
 };
@@ -266,21 +275,24 @@ __device__ __forceinline__ void raw_word(uint32_t w, uint32_t (&v)[4]) {
   v[3] = lop3_and_or(w8, 0x00F000F0u, 0x64006400u);
 }
 
-template <int kNTiles, bool kOffset>
-__global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
+template <int kNTiles, bool kOffset, int kCW>
+__global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
     const __grid_constant__ CUtensorMap tmap_z, const uint32_t* __restrict__ qweight,
     const __half* __restrict__ X, int M, int64_t N, int64_t K, const float* __restrict__ inv_s,
-    __half* __restrict__ Y, G4Smem lay) {
-  extern __shared__ __align__(128) uint8_t smem[];
+    __half* __restrict__ Y, G4Smem lay, unsigned flags) {
+  static_assert(kG4Groups % kCW == 0, "consumer warps must divide the unit's groups");
+  constexpr int kGPW = kG4Groups / kCW;   // groups per consumer warp and unit
   constexpr int kTok = 8 * kNTiles;
+  extern __shared__ __align__(128) uint8_t smem[];
   __half* xs = reinterpret_cast<__half*>(smem);
   float* cc = reinterpret_cast<float*>(smem + lay.c_off());
   uint8_t* slots = smem + lay.slot_off();
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bar_off());
-  uint64_t* empty = full + kG4Slots;
-  uint64_t* xfull = empty + kG4Slots;
+  uint64_t* empty = full + kGSMaxSlots;
+  uint64_t* xfull = empty + kGSMaxSlots;
   float* red = reinterpret_cast<float*>(smem + lay.red_off());
+  const int S = lay.slots;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -293,22 +305,41 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
   const int64_t units = (t1 - t0) * C;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kG4Slots; ++i) {
+    for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kG4Warps * 32);
+      mbar_init(&empty[i], kCW * 32);
     }
     mbar_init(xfull, 1);
     fence_barrier_init();
   }
   __syncthreads();
 
-  if (warp == kG4Warps) {
+  if (warp == kCW) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      pdl_launch_dependents();
       tma_prefetch_desc(&tmap_w);
       tma_prefetch_desc(&tmap_s);
       tma_prefetch_desc(&tmap_z);
+      int slot = 0, chunk = 0;
+      uint32_t ph = 0;
+      int64_t tile = t0;
+      auto issue = [&]() {
+        if (!AWQ_IN_BOUNDS(slot < S && tile < t1 && chunk < C)) return;
+        uint8_t* sb = slots + slot * kG4SlotBytes;
+        mbar_arrive_expect_tx(&full[slot], kG4SlotBytes);
+        const int32_t row = static_cast<int32_t>(tile * kGemvRows);
+        tma_load_2d(sb, &tmap_w, &full[slot], chunk * (kG4KC / 8), row);
+        tma_load_2d(sb + kG4WBytes, &tmap_s, &full[slot], row, chunk * kG4Groups);
+        tma_load_2d(sb + kG4WBytes + kG4SBytes, &tmap_z, &full[slot], row, chunk * kG4Groups);
+        if (++slot == S) { slot = 0; ph ^= 1; }
+        if (++chunk == C) { chunk = 0; ++tile; }
+      };
+      int64_t u = 0;
+      if (flags & kGemvWeightsReady) {
+        // the weights do not depend on the preceding kernel: fill the (empty) ring now
+        const int64_t n_early = units < S ? units : S;
+        for (; u < n_early; ++u) issue();
+      }
       {   // HBM -> L2 for this CTA's weight rows (one contiguous range)
         const int64_t row_bytes = K / 2;
         const int64_t r0 = t0 * kGemvRows, r1 = t1 * kGemvRows < N ? t1 * kGemvRows : N;
@@ -318,21 +349,13 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
           prefetch_l2_bulk(wrow + off, static_cast<uint32_t>(bytes - off < 65536 ? bytes - off : 65536));
       }
       pdl_wait();
+      // every kernel before this one has completed: the next grid may now be scheduled
+      pdl_launch_dependents();
       mbar_arrive_expect_tx(xfull, static_cast<uint32_t>(M * K * 2));
       bulk_load_1d(xs, X, static_cast<uint32_t>(M * K * 2), xfull);
-      int slot = 0, chunk = 0;
-      uint32_t ph = 0;
-      int64_t tile = t0;
-      for (int64_t u = 0; u < units; ++u) {
+      for (; u < units; ++u) {
         if (!mbar_wait(&empty[slot], ph ^ 1)) break;
-        uint8_t* sb = slots + slot * kG4SlotBytes;
-        mbar_arrive_expect_tx(&full[slot], kG4SlotBytes);
-        const int32_t row = static_cast<int32_t>(tile * kGemvRows);
-        tma_load_2d(sb, &tmap_w, &full[slot], chunk * (kG4KC / 8), row);
-        tma_load_2d(sb + kG4WBytes, &tmap_s, &full[slot], row, chunk * kG4Groups);
-        tma_load_2d(sb + kG4WBytes + kG4SBytes, &tmap_z, &full[slot], row, chunk * kG4Groups);
-        if (++slot == kG4Slots) { slot = 0; ph ^= 1; }
-        if (++chunk == C) { chunk = 0; ++tile; }
+        issue();
       }
     }
     return;
@@ -351,7 +374,7 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
     const int sub = lane & 7;
     const int npairs = G * M;
     const __half2 sixteenth = __float2half2_rn(0.0625f);
-    for (int base = warp * 4; base < npairs; base += kG4Warps * 4) {
+    for (int base = warp * 4; base < npairs; base += kCW * 4) {
       const int pr = base + (lane >> 3);
       const bool live = ok && pr < npairs;
       const int g = live ? pr / M : 0, m = live ? pr % M : 0;
@@ -389,13 +412,13 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
         cc[(g * kTok + m) * 2 + 1] = c2;
       }
     }
-    for (int i = threadIdx.x; i < G * kTok; i += kG4Warps * 32)
+    for (int i = threadIdx.x; i < G * kTok; i += kCW * 32)
       if (i % kTok >= M) { cc[2 * i] = 0.0f; cc[2 * i + 1] = 0.0f; }
-    named_bar_sync(1, kG4Warps * 32);
+    named_bar_sync(1, kCW * 32);
   } else if (inv_s != nullptr) {
     // x <- fp16(x * inv_s)
     const int n8 = M * Ki / 8;
-    for (int i = threadIdx.x; ok && i < n8; i += kG4Warps * 32) {
+    for (int i = threadIdx.x; ok && i < n8; i += kCW * 32) {
       uint4 v = reinterpret_cast<uint4*>(xs)[i];
       const int k = (i * 8) % Ki;
       const float4 s0 = *reinterpret_cast<const float4*>(inv_s + k);
@@ -407,7 +430,7 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
       f = __half22float2(u32_as_h2(v.w)); v.w = h2_as_u32(__floats2half2_rn(f.x * s1.z, f.y * s1.w));
       reinterpret_cast<uint4*>(xs)[i] = v;
     }
-    named_bar_sync(1, kG4Warps * 32);
+    named_bar_sync(1, kCW * 32);
   }
 
   float total[kNTiles][4];
@@ -421,18 +444,17 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
   int64_t tile = t0;
   for (int64_t u = 0; u < units; ++u) {
     ok = __all_sync(0xffffffffu, ok && mbar_wait(&full[slot], ph));
-    // Copy this warp's operands of the unit (two groups: packed words of rows r and r + 8,
+    // Copy this warp's operands of the unit (its groups: packed words of rows r and r + 8,
     // their scales and zero points) to registers and release the slot at once, so the
-    // producer refills it while this unit is computed: the ring then keeps its full depth
-    // of weight bytes in flight instead of holding a slot through the arithmetic. Every
-    // lane arrives (release semantics), which orders its own shared-memory reads first.
+    // producer refills it while this unit is computed. Every lane arrives (release
+    // semantics), which orders its own shared-memory reads first.
     const uint8_t* sb = slots + slot * kG4SlotBytes;
-    uint4 wA[2], wB[2];
-    uint32_t zAi[2], zBi[2];
-    float scA[2], scB[2];
+    uint4 wA[kGPW], wB[kGPW];
+    uint32_t zAi[kGPW], zBi[kGPW];
+    float scA[kGPW], scB[kGPW];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int gl = 2 * warp + q;               // group inside the unit
+    for (int q = 0; q < kGPW; ++q) {
+      const int gl = kGPW * warp + q;               // group inside the unit
       const uint8_t* wrow = sb + (gl * 16 + 4 * c) * 4;
       wA[q] = *reinterpret_cast<const uint4*>(wrow + r * (kG4KC / 2));
       wB[q] = *reinterpret_cast<const uint4*>(wrow + (r + 8) * (kG4KC / 2));
@@ -444,17 +466,19 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
       scB[q] = __half2float(ss[r + 8]);
     }
     if (ok) mbar_arrive(&empty[slot]);
-    if (++slot == kG4Slots) { slot = 0; ph ^= 1; }
+    if (++slot == S) { slot = 0; ph ^= 1; }
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int gl = 2 * warp + q;
+    for (int q = 0; q < kGPW; ++q) {
+      const int gl = kGPW * warp + q;
       const int g = chunk * kG4Groups + gl;
       if (ok && g < G) {
-        float acc[kNTiles][2][4];
+        float acc[kNTiles][4][4];
 #pragma unroll
         for (int t = 0; t < kNTiles; ++t)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) acc[t][0][i] = acc[t][1][i] = 0.0f;
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[t][j][i] = 0.0f;
         const uint32_t wordsA[4] = {wA[q].x, wA[q].y, wA[q].z, wA[q].w};
         const uint32_t wordsB[4] = {wB[q].x, wB[q].y, wB[q].z, wB[q].w};
         const int kx = g * kGroup + 32 * c;
@@ -479,19 +503,20 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
           for (int t = 0; t < kNTiles; ++t) {
             const int m = r + 8 * t;
             uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-            if (m < M) xv = *reinterpret_cast<const uint4*>(xs + m * Ki + kx + 8 * j);
+            if (m < M && AWQ_IN_BOUNDS(kx + 8 * j + 8 <= Ki))
+              xv = *reinterpret_cast<const uint4*>(xs + m * Ki + kx + 8 * j);
             const uint32_t a0[4] = {va[0], vb[0], va[1], vb[1]};
-            mma_16816(acc[t][j & 1], a0, xv.x, xv.y);
+            mma_16816(acc[t][j], a0, xv.x, xv.y);
             const uint32_t a1[4] = {va[2], vb[2], va[3], vb[3]};
-            mma_16816(acc[t][j & 1], a1, xv.z, xv.w);
+            mma_16816(acc[t][j], a1, xv.z, xv.w);
           }
         }
 #pragma unroll
         for (int t = 0; t < kNTiles; ++t) {
           float d[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) d[i] = acc[t][0][i] + acc[t][1][i];
-          if (kOffset) {
+          for (int i = 0; i < 4; ++i) d[i] = (acc[t][0][i] + acc[t][1][i]) + (acc[t][2][i] + acc[t][3][i]);
+          if (kOffset && AWQ_IN_BOUNDS((g * kTok + 8 * t + 2 * c) * 2 + 4 <= G * kTok * 2)) {
             const float zA = static_cast<float>(zAi[q]), zB = static_cast<float>(zBi[q]);
             const float4 cm = *reinterpret_cast<const float4*>(cc + (g * kTok + 8 * t + 2 * c) * 2);
             d[0] -= fmaf(zA, cm.y, cm.x);
@@ -508,7 +533,7 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
     }
 
     if (chunk == C - 1) {
-      // tile complete: fixed-order sum over the eight consumer warps, fp16 store
+      // tile complete: fixed-order sum over the consumer warps, fp16 store
 #pragma unroll
       for (int t = 0; t < kNTiles; ++t)
 #pragma unroll
@@ -516,7 +541,7 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
           red[((warp * kNTiles + t) * 4 + i) * 32 + lane] = total[t][i];
           total[t][i] = 0.0f;
         }
-      named_bar_sync(1, kG4Warps * 32);
+      named_bar_sync(1, kCW * 32);
       if (ok && warp < kNTiles) {
         const int t = warp;
         float v[4];
@@ -524,21 +549,21 @@ __global__ void __launch_bounds__(kG4Threads) gemv_stream_kernel(
         for (int i = 0; i < 4; ++i) {
           float sum = 0.0f;
 #pragma unroll
-          for (int w = 0; w < kG4Warps; ++w) sum += red[((w * kNTiles + t) * 4 + i) * 32 + lane];
+          for (int w = 0; w < kCW; ++w) sum += red[((w * kNTiles + t) * 4 + i) * 32 + lane];
           v[i] = sum;
         }
         const int64_t nA = tile * kGemvRows + r, nB = nA + 8;
         const int m0 = 8 * t + 2 * c, m1 = m0 + 1;
-        if (nA < N) {
+        if (nA < N && AWQ_IN_BOUNDS(tile < t1)) {
           if (m0 < M) Y[static_cast<int64_t>(m0) * N + nA] = __float2half_rn(v[0]);
           if (m1 < M) Y[static_cast<int64_t>(m1) * N + nA] = __float2half_rn(v[1]);
         }
-        if (nB < N) {
+        if (nB < N && AWQ_IN_BOUNDS(tile < t1)) {
           if (m0 < M) Y[static_cast<int64_t>(m0) * N + nB] = __float2half_rn(v[2]);
           if (m1 < M) Y[static_cast<int64_t>(m1) * N + nB] = __float2half_rn(v[3]);
         }
       }
-      named_bar_sync(1, kG4Warps * 32);
+      named_bar_sync(1, kCW * 32);
     }
     if (++chunk == C) { chunk = 0; ++tile; }
   }

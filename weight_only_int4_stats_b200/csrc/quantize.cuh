@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
       w0 |= q[o] << (4 * nibble_pos(o));
       w1 |= q[8 + o] << (4 * nibble_pos(o));
     }
-    if (valid)
+    if (valid && AWQ_IN_BOUNDS(j * 16 + 2 * sub + 2 <= K / 8))
       *reinterpret_cast<uint2*>(qweight + n * (K / 8) + j * 16 + 2 * sub) = make_uint2(w0, w1);
   } else {
     // lanes sub = 2b + h hold offsets 16h..16h+15 of the group's 32-k block b
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
       hi |= ((q[e] >> 2) & 1u) << ((o >> 1) + 16 * (o & 1));
     }
     hi |= __shfl_xor_sync(0xffffffffu, hi, 1);
-    if (valid) {
+    if (valid && AWQ_IN_BOUNDS((j * 4 + (sub >> 1)) * 3 + 3 <= 3 * K / 32)) {
       uint32_t* dst = qweight + n * (3 * K / 32) + (j * 4 + (sub >> 1)) * 3;
       dst[h] = lo;
       if (h == 0) dst[2] = hi;
@@ -160,8 +160,9 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
   __syncthreads();
   const int t = threadIdx.x;
   const int64_t nb = static_cast<int64_t>(blockIdx.x) * kQuantRowsPerCta;
-  if (t < kQuantRowsPerCta && nb + t < N) scales[j * N + nb + t] = sh_scale[t];
-  if (t >= 32 && t < 32 + kQuantRowsPerCta && nb + t - 32 < N)
+  const bool in_g = AWQ_IN_BOUNDS(j < K / kGroup);
+  if (t < kQuantRowsPerCta && nb + t < N && in_g) scales[j * N + nb + t] = sh_scale[t];
+  if (t >= 32 && t < 32 + kQuantRowsPerCta && nb + t - 32 < N && in_g)
     zeros[j * N + nb + t - 32] = sh_zero[t - 32];
 }
 
@@ -212,6 +213,7 @@ __global__ void __launch_bounds__(256) search_build_error_kernel(
     out[0] = make_uint4(e2[0], e2[1], e2[2], e2[3]);
     out[1] = make_uint4(e2[4], e2[5], e2[6], e2[7]);
   }
+  if (!AWQ_IN_BOUNDS(a < gridDim.z && k0 + 16 <= K)) return;
   uint4* dst = reinterpret_cast<uint4*>(E + a * N_pad * K + n * K + k0);
   dst[0] = out[0];
   dst[1] = out[1];

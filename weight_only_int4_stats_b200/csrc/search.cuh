@@ -21,7 +21,8 @@ __global__ void __launch_bounds__(kReduceThreads) search_row_loss_kernel(
   const int64_t rows_total = static_cast<int64_t>(n_alpha) * N_pad;
   const double* p = row_part + a * N_pad + n;
   double r = 0.0;
-  for (int j = 0; j < m_tiles; ++j) r += p[static_cast<int64_t>(j) * rows_total];
+  for (int j = 0; j < m_tiles; ++j)
+    if (AWQ_IN_BOUNDS(a * N_pad + n < rows_total)) r += p[static_cast<int64_t>(j) * rows_total];
   row_loss[i] = r;
 }
 
@@ -45,10 +46,13 @@ __global__ void __launch_bounds__(kReduceThreads) search_reduce_kernel(
 }
 
 // Every CTA finds the first minimum itself (n_alpha is small) and copies its slice of the
-// winning scale row; CTA 0 also writes the index.
+// winning scale row (and, when asked, of its correctly rounded reciprocal); CTA 0 also writes
+// the index.
 __global__ void search_pick_kernel(const double* __restrict__ losses, int n_alpha,
-                                   const float* __restrict__ s_table, int64_t K,
-                                   int32_t* __restrict__ best_idx, float* __restrict__ best_s) {
+                                   const float* __restrict__ s_table,
+                                   const float* __restrict__ inv_table, int64_t K,
+                                   int32_t* __restrict__ best_idx, float* __restrict__ best_s,
+                                   float* __restrict__ best_inv_s) {
   int best = 0;
   double bl = losses[0];
   for (int a = 1; a < n_alpha; ++a) {
@@ -57,24 +61,10 @@ __global__ void search_pick_kernel(const double* __restrict__ losses, int n_alph
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) best_idx[0] = best;
   const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (k < K) best_s[k] = s_table[static_cast<int64_t>(best) * K + k];
-}
-
-// x'[m, k] = fp16(x[m, k] * inv_s[k]) for the tensor-core GEMM's activation operand.
-__global__ void prescale_x_kernel(const __half* __restrict__ X, const float* __restrict__ inv_s,
-                                  int64_t M, int64_t K, __half* __restrict__ Xs) {
-  const int64_t i8 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
-  if (i8 >= M * K) return;
-  const int64_t k = i8 % K;
-  uint4 v = *reinterpret_cast<const uint4*>(X + i8);
-  const float4 s0 = *reinterpret_cast<const float4*>(inv_s + k);
-  const float4 s1 = *reinterpret_cast<const float4*>(inv_s + k + 4);
-  float2 f;
-  f = __half22float2(u32_as_h2(v.x)); v.x = h2_as_u32(__floats2half2_rn(f.x * s0.x, f.y * s0.y));
-  f = __half22float2(u32_as_h2(v.y)); v.y = h2_as_u32(__floats2half2_rn(f.x * s0.z, f.y * s0.w));
-  f = __half22float2(u32_as_h2(v.z)); v.z = h2_as_u32(__floats2half2_rn(f.x * s1.x, f.y * s1.y));
-  f = __half22float2(u32_as_h2(v.w)); v.w = h2_as_u32(__floats2half2_rn(f.x * s1.z, f.y * s1.w));
-  *reinterpret_cast<uint4*>(Xs + i8) = v;
+  if (k < K && AWQ_IN_BOUNDS(best >= 0 && best < n_alpha)) {
+    best_s[k] = s_table[static_cast<int64_t>(best) * K + k];
+    if (best_inv_s != nullptr) best_inv_s[k] = inv_table[static_cast<int64_t>(best) * K + k];
+  }
 }
 
 }  // namespace awq
