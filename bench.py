@@ -227,11 +227,14 @@ def capture_run(fn_per_step, first, count, stream):
 
 def time_steps(fn_per_step, steps, warmup, stream, world):
     """Warm-up graph of `warmup` steps, then a graph of exactly `steps` steps timed with
-    CUDA events on `stream`, with a barrier and a device synchronisation on both sides."""
+    CUDA events on `stream`, with a barrier and a device synchronisation on both sides. The
+    timed graph is also replayed once before the timed replay (its first replay uploads the
+    graph to the device), so the untimed warm-up is `warmup + steps` steps."""
     gw = capture_run(fn_per_step, 0, warmup, stream)
     gt = capture_run(fn_per_step, warmup, steps, stream)
     with torch.cuda.stream(stream):
         gw.replay()
+        gt.replay()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()

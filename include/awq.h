@@ -166,6 +166,20 @@ AWQ_API awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, cons
                             double* row_losses, void* workspace, size_t ws_bytes,
                             void* stream);
 
+/* ---------------------------------------------------------------- gated MLP calibration input
+ * robotsatlas.com "AWQ", "How it works": the calibration set is passed through the model, so
+ * each linear layer is calibrated on the activations that reach it. In a SiLU-gated MLP
+ * (this library's reading of the decoder layer's MLP) down_proj sees
+ *     H[m, i] = silu(g) * u,  g = sum_k X[m, k] W_gate[i, k],  u = sum_k X[m, k] W_up[i, k],
+ * silu(g) = g / (1 + exp(-g)), from the full-precision (fp16) gate_proj and up_proj weights.
+ * One tensor-core kernel computes both products of a 128-row tile (fp16 operands, fp32
+ * accumulation) and writes fp16 H.
+ * X: fp16 [M, K]; W_gate, W_up: fp16 [I, K]; H: fp16 [M, I] (output). K % 128 == 0.
+ * M = 0 or I = 0 is a no-op. No workspace. */
+AWQ_API awq_status awq_silu_mul_gemm(const awq_f16* X, int64_t M, const awq_f16* W_gate,
+                                     const awq_f16* W_up, int64_t I, int64_t K, awq_f16* H,
+                                     void* stream);
+
 /* ---------------------------------------------------------------- W4A16 GEMM
  * builderai.tools "AWQ", "About" (kernels for 4-bit weights with 16-bit activations);
  * robotsatlas.com "AWQ", "Implementation pitfalls" (dequantization fused into the GEMM).
@@ -186,11 +200,17 @@ AWQ_API awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, cons
  * weights loaded once): the decode kernel then starts streaming them at once, overlapping
  * the preceding kernel. X is always read only after the preceding kernel has completed.
  * (This library's kernels let the next launch start only after their own predecessor has
- * completed, so with them the window is exactly one kernel.) Other bits are rejected.
+ * completed, so with them the window is exactly one kernel.)
+ * AWQ_GEMM_BF16: X and Y are bf16 instead of fp16 (sourcepulse.org "AWQ", "Maintenance &
+ * Community": BF16 support); the packed weights, fp16 scales and zero points are the same.
+ * The decode kernels dequantize to exact (q - z) bf16 pairs and scale each group's fp32 sum;
+ * the tensor-core kernel feeds bf16 (q - z) * scale to the bf16 tensor cores. Other bits are
+ * rejected.
  * workspace: at least awq_gemm_workspace_size(M, N, K, bits) bytes: 0 unless the
  * tensor-core kernel splits K across CTAs (few output tiles), then room for the fp32
  * partial sums; the size does not depend on inv_s or flags. */
 #define AWQ_GEMM_WEIGHTS_READY 1u
+#define AWQ_GEMM_BF16 2u
 AWQ_API size_t awq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits);
 AWQ_API awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
                           const awq_f16* scales, const uint8_t* zeros, int64_t N, int64_t K,

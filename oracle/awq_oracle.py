@@ -60,6 +60,7 @@ __all__ = [
     "search_losses",
     "search_scale",
     "gemm_w4a16",
+    "silu_mul",
     "packed_words_per_row",
 ]
 
@@ -266,3 +267,20 @@ def gemm_w4a16(X, qweight, scales, zeros, N: int, K: int, bits: int, group: int,
     if inv_s is not None:
         x = x * np.asarray(inv_s, np.float32).astype(np.float64)[None, :]
     return x @ deq.T
+
+
+def silu_mul(X, W_gate, W_up):
+    """Input of a gated MLP's down projection: h = silu(g) * u with g = X W_gate^T,
+    u = X W_up^T and silu(g) = g / (1 + exp(-g)), all in fp64 from the fp16 operands.
+
+    robotsatlas "AWQ", "How it works": the calibration set is passed through the model, so each
+    linear layer is calibrated on the activations that actually reach it. In the 7B-shaped
+    decoder layer's MLP (a SiLU-gated MLP: this library's reading of the layer, which the
+    pages do not spell out) the activations reaching down_proj are this gated product of the
+    full-precision gate_proj and up_proj outputs.
+    """
+    x = np.asarray(X).astype(np.float64)
+    g = x @ np.asarray(W_gate).astype(np.float64).T
+    u = x @ np.asarray(W_up).astype(np.float64).T
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g)) * u

@@ -124,6 +124,20 @@ def _gemm_inv_s_ignored(X, qweight, scales, zeros, N, K, bits, group, inv_s=None
     return np.asarray(X).astype(np.float64) @ deq.T
 
 
+def _silu_mul_sign_slip(X, W_gate, W_up):
+    # exp(+g) in the logistic: g * sigmoid(-g) instead of g * sigmoid(g)
+    x = np.asarray(X).astype(np.float64)
+    g = x @ np.asarray(W_gate).astype(np.float64).T
+    u = x @ np.asarray(W_up).astype(np.float64).T
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(g)) * u
+
+
+def _silu_mul_gate_up_swapped(X, W_gate, W_up):
+    # the SiLU applied to up_proj's output instead of gate_proj's
+    return A.__dict__["_silu_mul_reference"](X, W_up, W_gate)
+
+
 MUTANTS = {
     "act_stats_abs_dropped": {"act_stats": _act_stats_no_abs},
     "act_stats_divides_by_m_minus_1": {"act_stats": _act_stats_m_minus_1},
@@ -145,6 +159,8 @@ MUTANTS = {
     "search_picks_largest_loss": {"search_scale": _search_scale_argmax},
     "search_ties_go_to_largest_alpha": {"search_scale": _search_scale_last_minimum},
     "gemm_ignores_inv_s": {"gemm_w4a16": _gemm_inv_s_ignored},
+    "silu_sign_slip": {"silu_mul": _silu_mul_sign_slip},
+    "silu_on_up_not_gate": {"silu_mul": _silu_mul_gate_up_swapped},
 }
 
 
@@ -152,6 +168,7 @@ def install(name: str) -> None:
     """Patch the named mutant into the oracle module and package."""
     if name == "none":
         return
+    A._silu_mul_reference = A.silu_mul   # the unmutated function, for mutants that wrap it
     for attr, fn in MUTANTS[name].items():
         assert hasattr(A, attr), attr
         setattr(A, attr, fn)

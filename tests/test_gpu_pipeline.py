@@ -93,3 +93,35 @@ def test_decoder_layer_pipeline_against_oracle(awq):
         err = rel_fro(Y.float().cpu().numpy(), want)
         assert err <= GEMM_RTOL, (n, err)
     torch.cuda.empty_cache()
+
+
+def test_down_proj_calibrated_on_gated_mlp_output(awq):
+    # down_proj's calibration input computed as a gated MLP would produce it: the GPU's
+    # H = silu(X W_gate^T) * (X W_up^T) from the hidden state's first 1024 tokens and the
+    # layer's fp16 gate_proj / up_proj against the oracle's; then down_proj's search on the
+    # oracle's H (fp16), GPU against oracle: s_x bit-exact, losses within the search
+    # tolerance, the same grid point (near ties aside), and the pack bit-exact.
+    X = synth.decoder_layer_activations(names=("hidden",), rows=TOKENS)["hidden"]
+    Ws = synth.decoder_layer_weights()
+    Wg, Wu, Wd = Ws["gate_proj"], Ws["up_proj"], Ws["down_proj"]
+    H = awq.awq_silu_mul_gemm(cu(X), cu(Wg), cu(Wu))
+    want = O.silu_mul(X, Wg, Wu)
+    assert rel_fro(H.float().cpu().numpy(), want) <= GEMM_RTOL
+    Hh = want.astype(np.float16)                  # the oracle's H feeds both searches
+    a = O.alpha_grid(20)
+    o_sx = O.act_stats(Hh)
+    ol, ob, obs = O.search_scale(Wd, Hh, o_sx, a, 4, 128)
+    Hd = cu(Hh)
+    sx = awq.awq_act_stats(Hd)
+    np.testing.assert_array_equal(sx.cpu().numpy(), o_sx)
+    losses, best, best_s, _ = awq.awq_search_scale(cu(Wd), Hd, sx, cu(a), 4)
+    np.testing.assert_allclose(losses.cpu().numpy(), ol, rtol=LOSS_RTOL)
+    b = int(best.item())
+    if b != ob:
+        assert ol[b] <= (1 + NEAR_TIE) * ol[ob], (b, ob)
+    gs = best_s.cpu().numpy()
+    qw, sc, z = awq.awq_quantize_pack(cu(Wd), best_s, 4)
+    oq, osc, oz = O.quantize_pack(Wd, gs, 4, 128)
+    np.testing.assert_array_equal(host_u32(qw), oq)
+    np.testing.assert_array_equal(z.cpu().numpy(), oz)
+    torch.cuda.empty_cache()

@@ -384,3 +384,74 @@ def test_gemm_brute_force_tiny():
             want = math.fsum(float(X[m, k]) * (int(codes[n, k]) - int(z[0, n])) * float(sc[0, n])
                              for k in range(K))
             assert abs(Y[m, n] - want) <= 1e-13 * max(1.0, abs(want))
+
+
+# ----------------------------------------------------------------------------- silu_mul
+
+def _select(rows, k):
+    """fp16 weight whose row i picks input channel rows[i] (a one-hot row), [len(rows), k]."""
+    W = np.zeros((len(rows), k), np.float16)
+    for i, c in enumerate(rows):
+        W[i, c] = 1.0
+    return W
+
+
+def test_silu_mul_closed_forms():
+    # One token whose channels hold g-values with closed-form SiLU: silu(0) = 0,
+    # silu(1) = e / (e + 1), silu(-1) = 1 / (e + 1) * -1, silu(ln 3) = (3/4) ln 3 (the logistic
+    # of ln 3 is 3/4), silu(-ln 3) = -(1/4) ln 3. W_gate selects channel i into output i; W_up
+    # selects the channel holding 1 (u = 1) or the channel holding 2 (u = 2).
+    ln3 = math.log(3.0)
+    e = math.e
+    gvals = [0.0, 1.0, -1.0, float(np.float16(ln3)), float(np.float16(-ln3))]
+    x = np.array([gvals + [1.0, 2.0]], np.float16)
+    K = x.shape[1]
+    Wg = _select(range(5), K)
+    h1 = O.silu_mul(x, Wg, _select([5] * 5, K))[0]
+    h2 = O.silu_mul(x, Wg, _select([6] * 5, K))[0]
+    l3 = gvals[3]
+    want = [0.0, e / (e + 1.0), -1.0 / (e + 1.0), l3 * 0.75, gvals[4] * 0.25]
+    # fp16(ln 3) is not ln 3: its logistic is 3/4 only to within |fp16(ln3) - ln3| / 4
+    tol = [1e-15, 1e-15, 1e-15, abs(l3 - ln3), abs(l3 - ln3)]
+    for got, w, t in zip(h1, want, tol):
+        assert abs(got - w) <= t + 1e-15
+    np.testing.assert_allclose(h2, 2.0 * h1, rtol=1e-15, atol=0)
+
+
+def test_silu_mul_odd_part_and_large_gates():
+    # silu(g) - silu(-g) = g for every g (the logistic satisfies s(g) + s(-g) = 1), and
+    # silu(g) -> g for large g, -> 0 for very negative g; u scales h linearly
+    rng = np.random.default_rng(7)
+    K = 64
+    x = (rng.standard_normal((16, K), dtype=np.float32) * 3).astype(np.float16)
+    Wg = (rng.standard_normal((24, K), dtype=np.float32) * 0.1).astype(np.float16)
+    zero_part = np.zeros((24, K), np.float16)
+    x1 = np.concatenate([x, np.ones((16, 1), np.float16)], axis=1)
+    Wg1 = np.concatenate([Wg, np.zeros((24, 1), np.float16)], axis=1)
+    Wu1 = np.concatenate([zero_part, np.ones((24, 1), np.float16)], axis=1)   # u = 1
+    hp = O.silu_mul(x1, Wg1, Wu1)
+    hn = O.silu_mul(x1, -Wg1, Wu1)
+    g = x1.astype(np.float64) @ Wg1.astype(np.float64).T
+    np.testing.assert_allclose(hp - hn, g, rtol=1e-12, atol=1e-12)
+    big = np.array([[60.0, 1.0]], np.float16)
+    Wbig = np.array([[1.0, 0.0], [-1.0, 0.0]], np.float16)
+    Wone = np.array([[0.0, 1.0], [0.0, 1.0]], np.float16)
+    hb = O.silu_mul(big, Wbig, Wone)[0]
+    assert abs(hb[0] - 60.0) < 1e-20 * 60 + 60 * math.exp(-60) * 1.01
+    assert 0.0 >= hb[1] > -60.0 * math.exp(-60) * 1.01
+    np.testing.assert_array_equal(O.silu_mul(x1, Wg1, np.zeros_like(Wu1)), 0.0)
+
+
+def test_silu_mul_brute_force_tiny():
+    rng = np.random.default_rng(8)
+    M, I, K = 3, 4, 40
+    x = rng.standard_normal((M, K), dtype=np.float32).astype(np.float16)
+    Wg = (rng.standard_normal((I, K), dtype=np.float32) * 0.3).astype(np.float16)
+    Wu = (rng.standard_normal((I, K), dtype=np.float32) * 0.3).astype(np.float16)
+    got = O.silu_mul(x, Wg, Wu)
+    for m in range(M):
+        for i in range(I):
+            g = math.fsum(float(x[m, k]) * float(Wg[i, k]) for k in range(K))
+            u = math.fsum(float(x[m, k]) * float(Wu[i, k]) for k in range(K))
+            want = g * u / (1.0 + math.exp(-g))
+            assert abs(got[m, i] - want) <= 1e-12 * (abs(want) + 1e-12)

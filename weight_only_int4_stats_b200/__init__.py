@@ -15,7 +15,8 @@ import torch
 __all__ = [
     "AwqError", "lib", "load_library", "library_path", "GROUP",
     "awq_act_stats", "awq_act_stats_noalloc", "awq_quantize_pack", "awq_search_scale", "awq_gemm_w4a16",
-    "awq_check_error", "packed_words_per_row", "WEIGHTS_READY",
+    "awq_silu_mul_gemm",
+    "awq_check_error", "packed_words_per_row", "WEIGHTS_READY", "BF16",
 ]
 
 GROUP = 128
@@ -59,6 +60,7 @@ def load_library(path: str) -> ctypes.CDLL:
         "awq_search_scale": (I32, [P, I64, I64, P, I64, P, P, I32, I32, I32, P, P, P, P, P,
                                    P, P, SZ, P]),
         "awq_gemm_workspace_size": (SZ, [I64, I64, I64, I32]),
+        "awq_silu_mul_gemm": (I32, [P, I64, P, P, I64, I64, P, P]),
         "awq_gemm_w4a16": (I32, [P, I64, P, P, P, I64, I64, I32, I32, P, ctypes.c_uint, P,
                                  P, SZ, P]),
     }
@@ -191,23 +193,27 @@ def awq_search_scale(W: torch.Tensor, X: torch.Tensor, s_x: torch.Tensor | None,
 
 
 WEIGHTS_READY = 1   # AWQ_GEMM_WEIGHTS_READY
+BF16 = 2            # AWQ_GEMM_BF16
 
 
 def awq_gemm_w4a16(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
                    zeros: torch.Tensor, N: int, K: int, bits: int = 4, group: int = GROUP,
                    inv_s: torch.Tensor | None = None, out: torch.Tensor | None = None,
                    workspace=None, stream=None, weights_ready: bool = False) -> torch.Tensor:
-    """Y = X deq(W)^T (fp16 [M, N]) with the dequantization fused into the kernel.
+    """Y = X deq(W)^T ([M, N], X's dtype) with the dequantization fused into the kernel.
 
-    ``weights_ready=True`` passes AWQ_GEMM_WEIGHTS_READY: the packed weights are not written
-    by the kernel launched just before this call on the stream, so the kernel may start
-    reading them while that kernel still runs."""
-    _need(X, torch.float16, "X")
+    X may be fp16 or bf16 (AWQ_GEMM_BF16); Y has X's dtype. ``weights_ready=True`` passes
+    AWQ_GEMM_WEIGHTS_READY: the packed weights are not written by the kernel launched just
+    before this call on the stream, so the kernel may start reading them while that kernel
+    still runs."""
+    bf16 = X.dtype == torch.bfloat16
+    _need(X, torch.bfloat16 if bf16 else torch.float16, "X")
     _need(scales, torch.float16, "scales")
     _need(zeros, torch.uint8, "zeros")
     _need(inv_s, torch.float32, "inv_s")
     M = X.shape[0]
-    Y = torch.empty(M, N, dtype=torch.float16, device=X.device) if out is None else out
+    Y = torch.empty(M, N, dtype=X.dtype, device=X.device) if out is None else out
+    _need(Y, X.dtype, "out")
     ws = workspace
     if ws is None:
         need = lib().awq_gemm_workspace_size(M, N, K, bits)
@@ -215,5 +221,24 @@ def awq_gemm_w4a16(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("awq_gemm_w4a16", lib().awq_gemm_w4a16(
         _ptr(X), M, _ptr(qweight), _ptr(scales), _ptr(zeros), N, K, bits, group, _ptr(inv_s),
-        WEIGHTS_READY if weights_ready else 0, _ptr(Y), _ptr(ws), ws_bytes, _stream(stream)))
+        (WEIGHTS_READY if weights_ready else 0) | (BF16 if bf16 else 0), _ptr(Y), _ptr(ws),
+        ws_bytes, _stream(stream)))
     return Y
+
+
+def awq_silu_mul_gemm(X: torch.Tensor, W_gate: torch.Tensor, W_up: torch.Tensor,
+                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H = silu(X W_gate^T) * (X W_up^T) (fp16 [M, I]): the input of a gated MLP's down
+    projection, computed from the full-precision weights for calibration."""
+    _need(X, torch.float16, "X")
+    _need(W_gate, torch.float16, "W_gate")
+    _need(W_up, torch.float16, "W_up")
+    M, K = X.shape
+    I = W_gate.shape[0]
+    if W_up.shape != W_gate.shape or W_gate.shape[1] != K:
+        raise ValueError("W_gate and W_up must both be [I, K]")
+    H = torch.empty(M, I, dtype=torch.float16, device=X.device) if out is None else out
+    _need(H, torch.float16, "out")
+    _check("awq_silu_mul_gemm", lib().awq_silu_mul_gemm(
+        _ptr(X), M, _ptr(W_gate), _ptr(W_up), I, K, _ptr(H), _stream(stream)))
+    return H

@@ -83,14 +83,14 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, in
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, ASrc kA, Epi kEpi>
-awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_rows,
-                     const awq::TcArgs& args, cudaStream_t st) {
+template <int BN, ASrc kA, Epi kEpi, bool kBf16 = false>
+awq_status launch_tc(const void* Xop, int64_t M, const void* Aop, int64_t a_rows,
+                     const awq::TcArgs& args, cudaStream_t st, const void* Aop2 = nullptr) {
   using L = awq::TcLayout<BN, kA>;
   static std::atomic<bool> attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
-  auto kern = awq::tc_gemm_kernel<BN, kA, kEpi>;
+  auto kern = awq::tc_gemm_kernel<BN, kA, kEpi, kBf16>;
   if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem) !=
         cudaSuccess)
@@ -98,10 +98,15 @@ awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_ro
     attr_set[dev].store(true, std::memory_order_release);
   }
   CUtensorMap tx, ta;
-  if (!make_tmap_2d(&tx, Xop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, args.K, BN, awq::kTcBK,
-                    true))
+  if (!make_tmap_2d(&tx, Xop, kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                    2, M, args.K, BN, awq::kTcBK, true))
     return AWQ_ERR_CUDA;
-  if (kA == ASrc::kFp16) {
+  if (kA == ASrc::kSplit16) {   // [a_rows, 2K]: the hi part, then the lo part, of each row
+    if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a_rows, 2 * args.K,
+                      awq::kTcBM, awq::kTcBK, true))
+      return AWQ_ERR_CUDA;
+  } else if (kA == ASrc::kPair16) {   // two [a_rows, K] weights; the second map goes in ts
     if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a_rows, args.K, awq::kTcBM,
                       awq::kTcBK, true))
       return AWQ_ERR_CUDA;
@@ -119,7 +124,11 @@ awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_ro
   CUtensorMap ts = ta, tz = ta;
   awq::TcArgs a = args;
   a.sz_tma = 0;
-  if (kA != ASrc::kFp16 && args.N % 16 == 0) {
+  if (kA == ASrc::kPair16 &&
+      !make_tmap_2d(&ts, Aop2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a_rows, args.K, awq::kTcBM,
+                    awq::kTcBK, true))
+    return AWQ_ERR_CUDA;
+  if ((kA == ASrc::kPacked4 || kA == ASrc::kPacked3) && args.N % 16 == 0) {
     const int64_t G = args.K / awq::kGroup;
     if (!make_tmap_2d(&ts, args.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, G, args.N, L::kPG,
                       awq::kTcBM, false) ||
@@ -149,13 +158,13 @@ awq_status launch_tc(const __half* Xop, int64_t M, const void* Aop, int64_t a_ro
   return launch_status();
 }
 
-template <ASrc kA, Epi kEpi>
-awq_status launch_tc_bn(const __half* Xop, int64_t M, const void* Aop, int64_t a_rows,
-                        const awq::TcArgs& args, cudaStream_t st) {
-  if (M <= 32) return launch_tc<32, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
-  if (M <= 64) return launch_tc<64, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
-  if (M <= 128) return launch_tc<128, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
-  return launch_tc<256, kA, kEpi>(Xop, M, Aop, a_rows, args, st);
+template <ASrc kA, Epi kEpi, bool kBf16 = false>
+awq_status launch_tc_bn(const void* Xop, int64_t M, const void* Aop, int64_t a_rows,
+                        const awq::TcArgs& args, cudaStream_t st, const void* Aop2 = nullptr) {
+  if (M <= 32) return launch_tc<32, kA, kEpi, kBf16>(Xop, M, Aop, a_rows, args, st, Aop2);
+  if (M <= 64) return launch_tc<64, kA, kEpi, kBf16>(Xop, M, Aop, a_rows, args, st, Aop2);
+  if (M <= 128) return launch_tc<128, kA, kEpi, kBf16>(Xop, M, Aop, a_rows, args, st, Aop2);
+  return launch_tc<256, kA, kEpi, kBf16>(Xop, M, Aop, a_rows, args, st, Aop2);
 }
 
 // Streaming decode GEMM (M <= 16, 4-bit), launched with programmatic dependent launch.
@@ -164,6 +173,7 @@ constexpr int kSmemLimit = 232448;   // 227 KB per CTA on sm_100
 constexpr int kCoResidentSmem = (233472 - 2 * 1024) / 2;
 
 static_assert(awq::kGemvWeightsReady == AWQ_GEMM_WEIGHTS_READY, "flag values must agree");
+static_assert((AWQ_GEMM_WEIGHTS_READY & AWQ_GEMM_BF16) == 0, "flags are distinct bits");
 
 struct GemvConfig {
   int cw;       // consumer warps (8 or 16)
@@ -200,15 +210,16 @@ bool gemv_stream_fits(int64_t M, int64_t N, int64_t K) {
   return gemv_config(M, N, K, 8, awq::kGSMaxSlots, 1, &c);
 }
 
-template <int kNTiles, bool kOffset, int kCW>
-awq_status launch_gemv_stream_cfg(const GemvConfig& cfgv, const __half* x, int64_t M,
+template <int kNTiles, bool kOffset, int kCW, bool kBf16 = false>
+awq_status launch_gemv_stream_cfg(const GemvConfig& cfgv, const void* x, int64_t M,
                                   const uint32_t* qweight, const __half* scales,
                                   const uint8_t* zeros, int64_t N, int64_t K, const float* inv_s,
-                                  unsigned flags, __half* y, cudaStream_t st) {
+                                  unsigned flags, void* y, cudaStream_t st) {
+  using A = awq::act_t<kBf16>;
   static std::atomic<bool> attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
-  auto kern = awq::gemv_stream_kernel<kNTiles, kOffset, kCW>;
+  auto kern = awq::gemv_stream_kernel<kNTiles, kOffset, kCW, kBf16>;
   if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
         cudaSuccess)
@@ -237,19 +248,29 @@ awq_status launch_gemv_stream_cfg(const GemvConfig& cfgv, const __half* x, int64
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int m32 = static_cast<int>(M);
-  if (cudaLaunchKernelEx(&cfg, kern, tw, ts, tz, qweight, x, m32, N, K, inv_s, y, cfgv.lay,
-                         flags) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kern, tw, ts, tz, qweight, static_cast<const A*>(x), m32, N, K,
+                         inv_s, static_cast<A*>(y), cfgv.lay, flags) != cudaSuccess)
     return AWQ_ERR_CUDA;
   return launch_status();
 }
 
 // Returns AWQ_ERR_UNSUPPORTED when the shape does not suit the streaming kernel; the caller
 // then uses the register-streaming kernel (M <= 8) or the tensor-core path.
-awq_status launch_gemv_stream(const __half* x, int64_t M, const uint32_t* qweight,
+awq_status launch_gemv_stream(const void* x, int64_t M, const uint32_t* qweight,
                               const __half* scales, const uint8_t* zeros, int64_t N, int64_t K,
-                              const float* inv_s, unsigned flags, __half* y, cudaStream_t st) {
+                              const float* inv_s, unsigned flags, void* y, cudaStream_t st) {
   GemvConfig c;
   if (!gemv_config(M, N, K, 8, awq::kGSMaxSlots, 1, &c)) return AWQ_ERR_UNSUPPORTED;
+  if (flags & AWQ_GEMM_BF16) {
+    if (M == 1)
+      return launch_gemv_stream_cfg<1, true, 8, true>(c, x, M, qweight, scales, zeros, N, K,
+                                                      inv_s, flags, y, st);
+    if (M <= 8)
+      return launch_gemv_stream_cfg<1, false, 8, true>(c, x, M, qweight, scales, zeros, N, K,
+                                                       inv_s, flags, y, st);
+    return launch_gemv_stream_cfg<2, false, 8, true>(c, x, M, qweight, scales, zeros, N, K,
+                                                     inv_s, flags, y, st);
+  }
   if (M == 1)
     return launch_gemv_stream_cfg<1, true, 8>(c, x, M, qweight, scales, zeros, N, K, inv_s,
                                               flags, y, st);
@@ -472,7 +493,7 @@ struct SearchWs {
 SearchWs search_ws_layout(int64_t M, int64_t N, int64_t K, int n_alpha) {
   const int64_t N_pad = round_up(N, awq::kTcBM);
   const int64_t m_tiles = (M + tc_bn_for(M) - 1) / tc_bn_for(M);
-  const size_t per_point = static_cast<size_t>(N_pad) * K * sizeof(__half);
+  const size_t per_point = static_cast<size_t>(N_pad) * 2 * K * sizeof(__half);   // hi, lo
   int64_t chunk = static_cast<int64_t>(kSearchChunkBytes / per_point);
   if (chunk < 1) chunk = 1;
   if (chunk > n_alpha) chunk = n_alpha;
@@ -562,7 +583,7 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
       args.row_part = part;
       args.m_tiles = m_tiles;
       args.k_splits = 1;
-      s = launch_tc_bn<ASrc::kFp16, Epi::kRowSumSq>(reinterpret_cast<const __half*>(X), M, E,
+      s = launch_tc_bn<ASrc::kSplit16, Epi::kRowSumSq>(X, M, E,
                                                     na * N_pad, args, st);
       if (s != AWQ_OK) return s;
     }
@@ -580,6 +601,30 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
   awq::search_pick_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(
       losses, n_alpha, S, inv, K, best_idx, best_s, best_inv_s);
   return launch_status();
+}
+
+// ------------------------------------------------------------------ gated MLP input
+awq_status awq_silu_mul_gemm(const awq_f16* X, int64_t M, const awq_f16* W_gate,
+                             const awq_f16* W_up, int64_t I, int64_t K, awq_f16* H,
+                             void* stream) {
+  if (bad_dim(M) || bad_dim(I) || bad_dim(K) || K == 0) return AWQ_ERR_INVALID_ARG;
+  if (K % awq::kGroup != 0) return AWQ_ERR_INVALID_ARG;
+  if (M == 0 || I == 0) return AWQ_OK;
+  if (!X || !W_gate || !W_up || !H) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(H))
+    return AWQ_ERR_INVALID_ARG;
+  if ((I + awq::kTcBM - 1) / awq::kTcBM > 65535) return AWQ_ERR_INVALID_ARG;
+  awq::TcArgs args{};
+  args.M = M;
+  args.N = I;
+  args.N_pad = I;
+  args.K = K;
+  args.Y = reinterpret_cast<__half*>(H);
+  args.m_tiles = static_cast<int>((M + tc_bn_for(M) - 1) / tc_bn_for(M));
+  args.k_splits = 1;
+  return launch_tc_bn<ASrc::kPair16, Epi::kSiluMul>(X, M,
+                                                    W_gate, I, args,
+                                                    static_cast<cudaStream_t>(stream), W_up);
 }
 
 // ------------------------------------------------------------------ GEMM
@@ -604,21 +649,22 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
   if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
       !aligned16(Y) || (inv_s && !aligned16(inv_s)))
     return AWQ_ERR_INVALID_ARG;
-  if ((flags & ~static_cast<unsigned>(AWQ_GEMM_WEIGHTS_READY)) != 0) return AWQ_ERR_INVALID_ARG;
+  if ((flags & ~static_cast<unsigned>(AWQ_GEMM_WEIGHTS_READY | AWQ_GEMM_BF16)) != 0)
+    return AWQ_ERR_INVALID_ARG;
+  const bool bf16 = (flags & AWQ_GEMM_BF16) != 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const __half* x = reinterpret_cast<const __half*>(X);
   const __half* sc = reinterpret_cast<const __half*>(scales);
-  __half* y = reinterpret_cast<__half*>(Y);
 
   if (M <= 16 && bits == 4) {
-    awq_status r = launch_gemv_stream(x, M, qweight, sc, zeros, N, K, inv_s, flags, y, st);
+    awq_status r = launch_gemv_stream(X, M, qweight, sc, zeros, N, K, inv_s, flags, Y, st);
     if (r != AWQ_ERR_UNSUPPORTED) return r;
-    // the streaming kernel cannot hold X (or N % 16 != 0): register streaming for M <= 8,
-    // the tensor-core path below for 8 < M <= 16
-    if (M <= 8) {
+    // the streaming kernel cannot hold X (or N % 16 != 0): register streaming for fp16 with
+    // M <= 8, the tensor-core path below otherwise
+    if (M <= 8 && !bf16) {
       const unsigned grid = static_cast<unsigned>((N + awq::kGemvRows - 1) / awq::kGemvRows);
       awq::gemv_w4a16_kernel<1><<<grid, awq::kGemvWarps * 32, 0, st>>>(
-          x, static_cast<int>(M), qweight, sc, zeros, N, K, inv_s, y);
+          reinterpret_cast<const __half*>(X), static_cast<int>(M), qweight, sc, zeros, N, K,
+          inv_s, reinterpret_cast<__half*>(Y));
       return launch_status();
     }
   }
@@ -636,18 +682,27 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
   args.K = K;
   args.scales = sc;
   args.zeros = zeros;
-  args.Y = y;
+  args.Y = Y;
   args.m_tiles = static_cast<int>((M + tc_bn_for(M) - 1) / tc_bn_for(M));
   args.k_splits = splits;
   args.partial = partial;
   args.inv_s = inv_s;   // folded into the dequantized weights by the builders
-  awq_status r =
-      bits == 3 ? launch_tc_bn<ASrc::kPacked3, Epi::kStoreY>(x, M, qweight, N, args, st)
-                : launch_tc_bn<ASrc::kPacked4, Epi::kStoreY>(x, M, qweight, N, args, st);
+  awq_status r;
+  if (bf16)
+    r = bits == 3 ? launch_tc_bn<ASrc::kPacked3, Epi::kStoreY, true>(X, M, qweight, N, args, st)
+                  : launch_tc_bn<ASrc::kPacked4, Epi::kStoreY, true>(X, M, qweight, N, args, st);
+  else
+    r = bits == 3 ? launch_tc_bn<ASrc::kPacked3, Epi::kStoreY>(X, M, qweight, N, args, st)
+                  : launch_tc_bn<ASrc::kPacked4, Epi::kStoreY>(X, M, qweight, N, args, st);
   if (r != AWQ_OK || splits == 1) return r;
   const int64_t MN = M * N;
-  awq::splitk_reduce_kernel<<<static_cast<unsigned>((MN / 4 + 1 + 255) / 256), 256, 0, st>>>(
-      partial, splits, MN, y);
+  const unsigned rgrid = static_cast<unsigned>((MN / 4 + 1 + 255) / 256);
+  if (bf16)
+    awq::splitk_reduce_kernel<true><<<rgrid, 256, 0, st>>>(
+        partial, splits, MN, reinterpret_cast<__nv_bfloat16*>(Y));
+  else
+    awq::splitk_reduce_kernel<false><<<rgrid, 256, 0, st>>>(partial, splits, MN,
+                                                            reinterpret_cast<__half*>(Y));
   return launch_status();
 }
 

@@ -4,9 +4,12 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 namespace awq {
 
@@ -273,10 +276,11 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
   return d;
 }
 
-// Instruction descriptor: fp16 A and B (both K-major), fp32 accumulator, M x N tile.
-__host__ __device__ constexpr uint32_t f16_idesc(int m, int n) {
-  return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
-         (static_cast<uint32_t>(m >> 4) << 24);
+// Instruction descriptor of kind::f16: fp16 (format 0) or bf16 (format 1) A and B, both
+// K-major, fp32 accumulator (D format 1), M x N tile.
+__host__ __device__ constexpr uint32_t f16_idesc(int m, int n, bool bf16 = false) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
+         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
 // ----------------------------------------------------------------------------- misc
@@ -300,6 +304,43 @@ __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
 }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
   return *reinterpret_cast<__half2*>(&u);
+}
+__device__ __forceinline__ uint32_t b2_as_u32(__nv_bfloat162 h) {
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ __nv_bfloat162 u32_as_b2(uint32_t u) {
+  return *reinterpret_cast<__nv_bfloat162*>(&u);
+}
+
+// 16-bit activations: fp16, or bf16 when kBf16 (the weights' scales stay fp16 in storage).
+template <bool kBf16>
+using act_t = std::conditional_t<kBf16, __nv_bfloat16, __half>;
+
+template <bool kBf16>
+__device__ __forceinline__ float2 act2_to_float2(uint32_t v) {
+  if constexpr (kBf16) return __bfloat1622float2(u32_as_b2(v));
+  else return __half22float2(u32_as_h2(v));
+}
+template <bool kBf16>
+__device__ __forceinline__ uint32_t float2_to_act2(float a, float b) {
+  if constexpr (kBf16) return b2_as_u32(__floats2bfloat162_rn(a, b));
+  else return h2_as_u32(__floats2half2_rn(a, b));
+}
+template <bool kBf16>
+__device__ __forceinline__ act_t<kBf16> float_to_act(float a) {
+  if constexpr (kBf16) return __float2bfloat16_rn(a);
+  else return __float2half_rn(a);
+}
+
+// Eight activations (one 16-byte chunk) times eight fp32 factors, rounded back to 16 bits.
+template <bool kBf16>
+__device__ __forceinline__ uint4 scale8(uint4 v, float4 s0, float4 s1) {
+  float2 f;
+  f = act2_to_float2<kBf16>(v.x); v.x = float2_to_act2<kBf16>(f.x * s0.x, f.y * s0.y);
+  f = act2_to_float2<kBf16>(v.y); v.y = float2_to_act2<kBf16>(f.x * s0.z, f.y * s0.w);
+  f = act2_to_float2<kBf16>(v.z); v.z = float2_to_act2<kBf16>(f.x * s1.x, f.y * s1.y);
+  f = act2_to_float2<kBf16>(v.w); v.w = float2_to_act2<kBf16>(f.x * s1.z, f.y * s1.w);
+  return v;
 }
 
 }  // namespace awq

@@ -12,7 +12,8 @@
 // order (see tile_of_block) with a shared-memory ring of 64-wide K stages that runs on
 // across tiles, and two TMEM accumulators so a tile's epilogue overlaps the next tile's
 // main loop:
-//   warp 5       TMA producer: X slice (128-byte swizzle), and the A slice (fp16 source);
+//   warp 5       TMA producer: X slice (128-byte swizzle), and both parts of the A slice
+//                (two-part fp16 source);
 //   warp 1       TMEM allocator and single-thread tcgen05.mma issuer (kind::f16, fp32 acc);
 //   warp 9       TMA producer of the packed source: kPG consecutive 128-k groups of packed
 //                weights (with their scales and zero points) per slot of a ring as deep as
@@ -52,15 +53,25 @@ constexpr int kTcEpiWarp0 = 12;   // warps 12..15: TMEM lane quarters 0..3 (warp
 constexpr int kTcPkSlotsMax = 16;   // deepest packed ring
 constexpr int kTcSmemMax = 232448;  // dynamic shared memory per CTA on sm_100
 
-enum class ASrc : int { kPacked4 = 0, kPacked3 = 1, kFp16 = 2 };
-enum class Epi : int { kStoreY = 0, kRowSumSq = 1 };
+// kSplit16: the search's error operand in two fp16 parts, E = hi + 2^-12 lo, stored as one
+// [rows, 2K] matrix (hi in columns 0..K-1, lo in K..2K-1); each part has its own accumulator
+// and the epilogue combines them in fp32.
+// kPair16: two fp16 weights of the same shape (a gated MLP's gate_proj and up_proj); the
+// same rows of both are the two A parts, each with its own accumulator.
+enum class ASrc : int { kPacked4 = 0, kPacked3 = 1, kSplit16 = 2, kPair16 = 3 };
+// kStoreY: fp16 Y (or fp32 split-K partials); kRowSumSq: per-row sums of squares of the
+// recombined two-part product; kSiluMul: fp16 H = silu(D_0) * D_1 of the two accumulators.
+enum class Epi : int { kStoreY = 0, kRowSumSq = 1, kSiluMul = 2 };
 
 template <int BN, ASrc kA>
 struct TcLayout {
-  static constexpr bool kPk = kA != ASrc::kFp16;
-  static constexpr int kStages = !kPk ? (BN >= 256 ? 4 : 6) : (BN >= 256 ? 4 : BN >= 64 ? 5 : 6);
+  static constexpr bool kPk = kA == ASrc::kPacked4 || kA == ASrc::kPacked3;
+  static constexpr int kStages =
+      !kPk ? (BN >= 256 ? 3 : BN >= 128 ? 4 : BN >= 64 ? 5 : 6) : (BN >= 256 ? 4 : BN >= 64 ? 5 : 6);
   static constexpr int kXBytes = BN * kTcBK * 2;
-  static constexpr int kABytes = kTcBM * kTcBK * 2;
+  static constexpr int kAParts = kPk ? 1 : 2;            // A tiles (and accumulators) per stage
+  static constexpr int kAPartBytes = kTcBM * kTcBK * 2;
+  static constexpr int kABytes = kAParts * kAPartBytes;
   // packed source: kPG groups (2 kPG stages) per ring slot
   static constexpr int kPG = !kPk ? 1 : BN <= 64 ? 4 : BN <= 128 ? 2 : 1;
   static constexpr int kPGroupBytes = kA == ASrc::kPacked4 ? 64 : kA == ASrc::kPacked3 ? 48 : 0;
@@ -73,7 +84,7 @@ struct TcLayout {
   static constexpr int kPFit =
       (kTcSmemMax - 1024 - 512 - kStages * (kXBytes + kABytes)) / (kPBytes + kSZBytes);
   static constexpr int kPSlots =
-      kA == ASrc::kFp16 ? 0 : (kPFit < kTcPkSlotsMax ? kPFit : kTcPkSlotsMax);
+      !kPk ? 0 : (kPFit < kTcPkSlotsMax ? kPFit : kTcPkSlotsMax);
   static constexpr int kPBars = kPSlots > 0 ? kPSlots : 1;   // barrier pairs of the ring
   static constexpr int kXOff = 0;
   static constexpr int kAOff = kXOff + kStages * kXBytes;
@@ -83,8 +94,11 @@ struct TcLayout {
   // full[S], empty[S], built[S], pfull[P], pempty[P], acc_full[2], acc_empty[2], tmem slot
   static constexpr int kBytes = kBarOff + (3 * kStages + 2 * kPBars + 4) * 8 + 16;
   static constexpr int kSmem = kBytes + 1024;   // slack for 1024-byte alignment
-  static constexpr uint32_t kTxBytes = kXBytes + (kA == ASrc::kFp16 ? kABytes : 0);
-  static constexpr uint32_t kTmemCols = 2 * BN;   // two fp32 accumulators (power of 2)
+  static constexpr uint32_t kTxBytes = kXBytes + (kPk ? 0 : kABytes);
+  // one accumulator per A part, double-buffered when TMEM's 512 columns allow (so a tile's
+  // epilogue overlaps the next tile's main loop); a power of 2 of at least 32 columns
+  static constexpr int kAccBufs = 2 * kAParts * BN <= 512 ? 2 : 1;
+  static constexpr uint32_t kTmemCols = kAccBufs * kAParts * BN;
 };
 
 struct TcArgs {
@@ -94,7 +108,7 @@ struct TcArgs {
   int64_t K;
   const __half* scales; // [K/128, N] (packed source)
   const uint8_t* zeros; // [K/128, N]
-  __half* Y;            // [M, N] (store epilogue)
+  void* Y;              // [M, N] fp16 (bf16 with bf16 activations): Y or the SiLU output H
   double* row_part;     // [m_tiles, rows_total] (search epilogue)
   int m_tiles;
   int row_tiles;        // 128-row tiles of the A matrix
@@ -159,39 +173,55 @@ __device__ __forceinline__ uint4 dequant_word_scaled(uint32_t w, __half2 bias_lo
 }
 
 // The four scale pairs of 8 consecutive k starting at k0: fp16(sc * inv_s[k]) pairs, or sc
-// broadcast when inv_s is NULL. Folding inv_s into the weights computes
-// sum_k x[k] * (inv_s[k] * deq[k]) = sum_k (x[k] * inv_s[k]) * deq[k].
-__device__ __forceinline__ uint4 pair_scales(float sc, __half2 sc2, const float* inv_s,
+// broadcast when inv_s is NULL (bf16 pairs for bf16 activations). Folding inv_s into the
+// weights computes sum_k x[k] * (inv_s[k] * deq[k]) = sum_k (x[k] * inv_s[k]) * deq[k].
+template <bool kBf16 = false>
+__device__ __forceinline__ uint4 pair_scales(float sc, uint32_t sc2, const float* inv_s,
                                              int64_t k0) {
-  if (inv_s == nullptr) {
-    const uint32_t s = h2_as_u32(sc2);
-    return make_uint4(s, s, s, s);
-  }
+  if (inv_s == nullptr) return make_uint4(sc2, sc2, sc2, sc2);
   const float4 a = *reinterpret_cast<const float4*>(inv_s + k0);
   const float4 b = *reinterpret_cast<const float4*>(inv_s + k0 + 4);
-  return make_uint4(h2_as_u32(__floats2half2_rn(sc * a.x, sc * a.y)),
-                    h2_as_u32(__floats2half2_rn(sc * a.z, sc * a.w)),
-                    h2_as_u32(__floats2half2_rn(sc * b.x, sc * b.y)),
-                    h2_as_u32(__floats2half2_rn(sc * b.z, sc * b.w)));
+  return make_uint4(float2_to_act2<kBf16>(sc * a.x, sc * a.y),
+                    float2_to_act2<kBf16>(sc * a.z, sc * a.w),
+                    float2_to_act2<kBf16>(sc * b.x, sc * b.y),
+                    float2_to_act2<kBf16>(sc * b.z, sc * b.w));
+}
+
+// bf16 form of the 4-bit dequantization: the exact (q - z) pairs (raw 128 + q minus the bias
+// pair 128 + z) times the scale pairs, one bf16 rounding of each product.
+__device__ __forceinline__ uint4 dequant_word_scaled_bf16(uint32_t w, uint32_t bias, uint4 c) {
+  const uint32_t v[4] = {lop3_and_or(w, 0x000F000Fu, 0x43004300u),
+                         lop3_and_or(w >> 4, 0x000F000Fu, 0x43004300u),
+                         lop3_and_or(w >> 8, 0x000F000Fu, 0x43004300u),
+                         lop3_and_or(w >> 12, 0x000F000Fu, 0x43004300u)};
+  const uint32_t cc[4] = {c.x, c.y, c.z, c.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    o[i] = b2_as_u32(__hmul2(__hsub2(u32_as_b2(v[i]), u32_as_b2(bias)), u32_as_b2(cc[i])));
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // 3-bit: the fp16 pair (q - z) * sc for k-offsets (2e, 2e+1) of chunk i (k = 8i..8i+7) of a
 // 32-k block whose low-bit words are w0 (offsets 0..15) / w1 (16..31) and whose bit-2 word
 // is w2 (the pair's two bits sit at bits hb and hb + 16; both are moved to bit 2 of their
 // 16-bit half by a single shift whose direction is fixed at compile time).
-template <int kI, int kE>
+template <int kI, int kE, bool kBf16 = false>
 __device__ __forceinline__ uint32_t dequant3_pair(uint32_t w0, uint32_t w1, uint32_t w2,
-                                                  __half2 bias_lo, uint32_t sc2u) {
-  const __half2 sc2 = u32_as_h2(sc2u);
+                                                  uint32_t bias_lo, uint32_t sc2u) {
   constexpr int pp = 4 * (kI & 1) + kE;     // 2-bit field of the pair inside its low word
   constexpr int hb = 4 * kI + kE;           // bit of the pair inside the bit-2 word
   const uint32_t wlo = (kI < 2) ? w0 : w1;
-  const uint32_t lo = lop3_and_or(wlo >> (2 * pp), 0x00030003u, 0x64006400u);
+  // 1024 + q in fp16 (0x6400), 128 + q in bf16 (0x4300): q in the low mantissa bits
+  const uint32_t lo = lop3_and_or(wlo >> (2 * pp), 0x00030003u, kBf16 ? 0x43004300u : 0x64006400u);
   const uint32_t hs = hb >= 2 ? (w2 >> (hb >= 2 ? hb - 2 : 0)) : (w2 << (hb < 2 ? 2 - hb : 0));
   uint32_t v;
   // (hs & 0x00040004) | lo
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(v) : "r"(hs), "r"(0x00040004u), "r"(lo));
-  return h2_as_u32(__hmul2(__hsub2(u32_as_h2(v), bias_lo), sc2));
+  if constexpr (kBf16)
+    return b2_as_u32(__hmul2(__hsub2(u32_as_b2(v), u32_as_b2(bias_lo)), u32_as_b2(sc2u)));
+  else
+    return h2_as_u32(__hmul2(__hsub2(u32_as_h2(v), u32_as_h2(bias_lo)), u32_as_h2(sc2u)));
 }
 
 // Byte offset of 16-byte chunk c (k = 8c..8c+7) of row r in a 64-wide fp16 tile stored in
@@ -200,7 +230,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
   return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
 
-template <int BN, ASrc kA, Epi kEpi>
+template <int BN, ASrc kA, Epi kEpi, bool kBf16 = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                    const __grid_constant__ CUtensorMap tmap_a,
@@ -208,7 +238,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    const __grid_constant__ CUtensorMap tmap_z, const TcArgs args) {
   using L = TcLayout<BN, kA>;
   constexpr int S = L::kStages;
-  constexpr bool kPacked = kA != ASrc::kFp16;
+  constexpr bool kPacked = L::kPk;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -218,6 +248,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* pfull = built + S;
   constexpr int P = L::kPBars;
   static_assert(!kPacked || L::kPSlots >= 2, "packed ring needs two slots");
+  static_assert(kEpi != Epi::kRowSumSq || kA == ASrc::kSplit16,
+                "the sum-of-squares epilogue recombines the two-part error operand");
+  static_assert(kEpi != Epi::kSiluMul || kA == ASrc::kPair16,
+                "the SiLU epilogue combines the gate and up accumulators");
+  static_assert(kEpi != Epi::kStoreY || kPacked, "fp16 Y comes from the packed sources");
   static_assert(L::kSmem <= kTcSmemMax, "shared memory layout too large");
   uint64_t* pempty = pfull + P;
   uint64_t* acc_full = pempty + P;
@@ -250,6 +285,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tma_prefetch_desc(&tmap_s);
       tma_prefetch_desc(&tmap_z);
     }
+    if (kA == ASrc::kPair16) tma_prefetch_desc(&tmap_s);
   }
   if (warp == kTcMmaWarp) {
     tmem_alloc(tmem_slot, L::kTmemCols);
@@ -285,9 +321,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           mbar_arrive_expect_tx(&full[s], L::kTxBytes);
           tma_load_2d(smem + L::kXOff + s * L::kXBytes, &tmap_x, &full[s], kb * kTcBK,
                       static_cast<int32_t>(m0));
-          if (kA == ASrc::kFp16)
-            tma_load_2d(smem + L::kAOff + s * L::kABytes, &tmap_a, &full[s], kb * kTcBK,
+          if (kA == ASrc::kSplit16) {
+            uint8_t* a = smem + L::kAOff + s * L::kABytes;
+            tma_load_2d(a, &tmap_a, &full[s], kb * kTcBK, static_cast<int32_t>(row0));
+            tma_load_2d(a + L::kAPartBytes, &tmap_a, &full[s],
+                        static_cast<int32_t>(args.K) + kb * kTcBK, static_cast<int32_t>(row0));
+          } else if (kA == ASrc::kPair16) {   // gate rows, then the same rows of up
+            uint8_t* a = smem + L::kAOff + s * L::kABytes;
+            tma_load_2d(a, &tmap_a, &full[s], kb * kTcBK, static_cast<int32_t>(row0));
+            tma_load_2d(a + L::kAPartBytes, &tmap_s, &full[s], kb * kTcBK,
                         static_cast<int32_t>(row0));
+          }
           if (++s == S) { s = 0; ph ^= 1; }
         }
       }
@@ -295,18 +339,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == kTcMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = f16_idesc(kTcBM, BN);
+      constexpr uint32_t idesc = f16_idesc(kTcBM, BN, kBf16);
       int s = 0;
       uint32_t ph = 0;
       int64_t lt = 0;
       bool ok = true;
       for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x, ++lt) {
         const TcUnit t = unit_of(u, args);
-        const int buf = static_cast<int>(lt & 1);
-        const uint32_t acc_ph = static_cast<uint32_t>((lt >> 1) & 1);
+        const int buf = static_cast<int>(lt % L::kAccBufs);
+        const uint32_t acc_ph = static_cast<uint32_t>((lt / L::kAccBufs) & 1);
         if (!mbar_wait(&acc_empty[buf], acc_ph ^ 1)) break;   // epilogue released the buffer
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * L::kAParts * BN);
         for (int i = 0; i < t.nkb; ++i) {
           ok = mbar_wait(&full[s], ph);
           if (ok && kPacked) ok = mbar_wait(&built[s], ph);
@@ -316,8 +360,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t x_base = smem_u32(smem + L::kXOff + s * L::kXBytes);
 #pragma unroll
           for (int kk = 0; kk < kTcBK / 16; ++kk) {
-            tc_mma_f16(d_tmem, sw128_kmajor_desc(a_base + kk * 32),
-                       sw128_kmajor_desc(x_base + kk * 32), idesc, (i | kk) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int part = 0; part < L::kAParts; ++part)   // part p: A tile p -> accumulator p
+              tc_mma_f16(d_tmem + static_cast<uint32_t>(part * BN),
+                         sw128_kmajor_desc(a_base + part * L::kAPartBytes + kk * 32),
+                         sw128_kmajor_desc(x_base + kk * 32), idesc, (i | kk) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[s]);
           if (++s == S) { s = 0; ph ^= 1; }
@@ -371,8 +418,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           const __half2 lo = u32_as_h2((0x6400u | z) * 0x00010001u);
           const __half2 hi = u32_as_h2((0xD400u | (z << 4)) * 0x00010001u);
-          const __half2 sc = __half2half2(sv);
           const float scf = __half2float(sv);
+          // the scale pair, and the bias pair 1024 + z (fp16) or 128 + z (bf16)
+          const uint32_t sc = kBf16 ? float2_to_act2<true>(scf, scf) : h2_as_u32(__half2half2(sv));
+          const uint32_t bias = kBf16 ? (0x4300u | z) * 0x00010001u : h2_as_u32(lo);
           const uint8_t* prow = smem + L::kPOff + ps * L::kPBytes + r * L::kPRowBytes;
 #pragma unroll
           for (int e = 0; e < 2; ++e) {             // stage i + e of the group
@@ -384,8 +433,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const int64_t k0 = static_cast<int64_t>(kb + e) * kTcBK + 32 * h + 8 * q;
-                const uint4 c4 = pair_scales(scf, sc, args.inv_s, k0);
-                const uint4 o = dequant_word_scaled(words[q], lo, hi, c4);
+                const uint4 c4 = pair_scales<kBf16>(scf, sc, args.inv_s, k0);
+                const uint4 o = kBf16 ? dequant_word_scaled_bf16(words[q], bias, c4)
+                                      : dequant_word_scaled(words[q], lo, hi, c4);
                 *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + q)) = o;
               }
             } else {
@@ -394,12 +444,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const uint32_t w0 = pw[0], w1 = pw[1], w2 = pw[2];
               uint4 o, c4;
 #define AWQ_DQ3_CHUNK(I)                                                                    \
-  c4 = pair_scales(scf, sc, args.inv_s,                                                    \
-                   static_cast<int64_t>(kb + e) * kTcBK + 32 * h + 8 * (I));               \
-  o.x = dequant3_pair<I, 0>(w0, w1, w2, lo, c4.x);                                         \
-  o.y = dequant3_pair<I, 1>(w0, w1, w2, lo, c4.y);                                         \
-  o.z = dequant3_pair<I, 2>(w0, w1, w2, lo, c4.z);                                         \
-  o.w = dequant3_pair<I, 3>(w0, w1, w2, lo, c4.w);                                         \
+  c4 = pair_scales<kBf16>(scf, sc, args.inv_s,                                             \
+                          static_cast<int64_t>(kb + e) * kTcBK + 32 * h + 8 * (I));        \
+  o.x = dequant3_pair<I, 0, kBf16>(w0, w1, w2, bias, c4.x);                                \
+  o.y = dequant3_pair<I, 1, kBf16>(w0, w1, w2, bias, c4.y);                                \
+  o.z = dequant3_pair<I, 2, kBf16>(w0, w1, w2, bias, c4.z);                                \
+  o.w = dequant3_pair<I, 3, kBf16>(w0, w1, w2, bias, c4.w);                                \
   *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + I)) = o;
               AWQ_DQ3_CHUNK(0)
               AWQ_DQ3_CHUNK(1)
@@ -430,17 +480,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x, ++lt) {
       const TcUnit t = unit_of(u, args);
-      const int buf = static_cast<int>(lt & 1);
-      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], static_cast<uint32_t>((lt >> 1) & 1)));
+      const int buf = static_cast<int>(lt % L::kAccBufs);
+      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf],
+                                             static_cast<uint32_t>((lt / L::kAccBufs) & 1)));
       if (!ok) break;
       tc_fence_after();
       const int64_t m0 = static_cast<int64_t>(t.m_tile) * BN;
       const int64_t arow = static_cast<int64_t>(t.row_tile) * kTcBM + row;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * wq) << 16) +
-                             static_cast<uint32_t>(buf * BN);
-      const bool unit_ok = AWQ_IN_BOUNDS(t.row_tile < args.row_tiles && t.m_tile < args.m_tiles &&
-                                         t.ksplit < args.k_splits &&
-                                         (buf + 1) * BN <= static_cast<int>(L::kTmemCols));
+                             static_cast<uint32_t>(buf * L::kAParts * BN);
+      const bool unit_ok =
+          AWQ_IN_BOUNDS(t.row_tile < args.row_tiles && t.m_tile < args.m_tiles &&
+                        t.ksplit < args.k_splits &&
+                        (buf + 1) * L::kAParts * BN <= static_cast<int>(L::kTmemCols));
       double sumsq = 0.0;
 #pragma unroll 1
       for (int col = 0; col < BN; col += 16) {
@@ -453,7 +505,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
                 const int64_t m = m0 + col + j;
-                if (m < args.M) args.Y[m * args.N + arow] = __float2half_rn(__uint_as_float(v[j]));
+                if (m < args.M)
+                  static_cast<act_t<kBf16>*>(args.Y)[m * args.N + arow] =
+                      float_to_act<kBf16>(__uint_as_float(v[j]));
               }
             } else {
               float* P = args.partial + static_cast<int64_t>(t.ksplit) * args.M * args.N;
@@ -464,11 +518,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               }
             }
           }
+        } else if (kEpi == Epi::kSiluMul) {
+          // h = silu(g) * u = g * u / (1 + exp(-g)), g and u the gate and up accumulators
+          uint32_t vu[16];
+          tmem_ld_32x32b_x16(taddr + BN + col, vu);
+          tmem_ld_wait();
+          if (arow < args.N && unit_ok) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int64_t m = m0 + col + j;
+              const float g = __uint_as_float(v[j]);
+              const float h = __fdiv_rn(g * __uint_as_float(vu[j]), 1.0f + expf(-g));
+              if (m < args.M) static_cast<__half*>(args.Y)[m * args.N + arow] = __float2half_rn(h);
+            }
+          }
         } else {
+          // D = D_hi + 2^-12 D_lo, the error operand's two parts recombined in fp32
+          uint32_t vl[16];
+          tmem_ld_32x32b_x16(taddr + BN + col, vl);
+          tmem_ld_wait();
           float part = 0.0f;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float f = __uint_as_float(v[j]);
+            const float f = fmaf(__uint_as_float(vl[j]), 0x1p-12f, __uint_as_float(v[j]));
             part = fmaf(f, f, part);
           }
           sumsq += static_cast<double>(part);
@@ -518,9 +590,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-// Y[m, n] = fp16(sum over the K slices of the fp32 partial sums), slices added in order.
+// Y[m, n] = fp16 (bf16) of the sum over the K slices of the fp32 partial sums, slices added
+// in order.
+template <bool kBf16 = false>
 __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int k_splits,
-                                     int64_t MN, __half* __restrict__ Y) {
+                                     int64_t MN, act_t<kBf16>* __restrict__ Y) {
   const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
   if (i >= MN) return;
   if ((MN & 3) == 0) {   // every slice's start is 16-byte aligned
@@ -530,14 +604,14 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int k_sp
       const float4 v = *reinterpret_cast<const float4*>(partial + static_cast<int64_t>(s) * MN + i);
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
-    *reinterpret_cast<__half2*>(Y + i) = __floats2half2_rn(acc.x, acc.y);
-    *reinterpret_cast<__half2*>(Y + i + 2) = __floats2half2_rn(acc.z, acc.w);
+    *reinterpret_cast<uint32_t*>(Y + i) = float2_to_act2<kBf16>(acc.x, acc.y);
+    *reinterpret_cast<uint32_t*>(Y + i + 2) = float2_to_act2<kBf16>(acc.z, acc.w);
   } else {   // this thread's four outputs, one at a time
     const int64_t end = i + 4 < MN ? i + 4 : MN;
     for (int64_t e = i; e < end; ++e) {
       float acc = partial[e];
       for (int s = 1; s < k_splits; ++s) acc += partial[static_cast<int64_t>(s) * MN + e];
-      Y[e] = __float2half_rn(acc);
+      Y[e] = float_to_act<kBf16>(acc);
     }
   }
 }

@@ -26,13 +26,21 @@ constexpr int kGemvWarps = 8;
 constexpr int kGemvRows = 16;
 constexpr int kGemvPrefetch = 4;   // groups of loads in flight per warp
 
+template <bool kBf16 = false>
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                           uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  if constexpr (kBf16)
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // Four fp16 pairs (q-z) from one packed word: pairs (k0,k1), (k2,k3), (k4,k5), (k6,k7).
@@ -266,26 +274,43 @@ struct G4Smem {
 };
 
 // One packed word -> the raw fp16 pairs (1024+q0,1024+q1), (1024+16q2,1024+16q3),
-// (1024+q4,1024+q5), (1024+16q6,1024+16q7).
+// (1024+q4,1024+q5), (1024+16q6,1024+16q7); with bf16 activations the raw bf16 pairs
+// (128+q0,128+q1), (128+q2,128+q3), ... (bf16 keeps only 7 mantissa bits, so each nibble
+// pair is shifted down first: 0x4300 is 128.0 and the low 4 mantissa bits hold q exactly).
+template <bool kBf16 = false>
 __device__ __forceinline__ void raw_word(uint32_t w, uint32_t (&v)[4]) {
-  const uint32_t w8 = w >> 8;
-  v[0] = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
-  v[1] = lop3_and_or(w, 0x00F000F0u, 0x64006400u);
-  v[2] = lop3_and_or(w8, 0x000F000Fu, 0x64006400u);
-  v[3] = lop3_and_or(w8, 0x00F000F0u, 0x64006400u);
+  if constexpr (kBf16) {
+    v[0] = lop3_and_or(w, 0x000F000Fu, 0x43004300u);
+    v[1] = lop3_and_or(w >> 4, 0x000F000Fu, 0x43004300u);
+    v[2] = lop3_and_or(w >> 8, 0x000F000Fu, 0x43004300u);
+    v[3] = lop3_and_or(w >> 12, 0x000F000Fu, 0x43004300u);
+  } else {
+    const uint32_t w8 = w >> 8;
+    v[0] = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
+    v[1] = lop3_and_or(w, 0x00F000F0u, 0x64006400u);
+    v[2] = lop3_and_or(w8, 0x000F000Fu, 0x64006400u);
+    v[3] = lop3_and_or(w8, 0x00F000F0u, 0x64006400u);
+  }
 }
 
-template <int kNTiles, bool kOffset, int kCW>
+// The exact pairs (q - z) in bf16: the raw pairs minus (128 + z).
+__device__ __forceinline__ void dequant_word_qz_bf16(uint32_t w, uint32_t bias, uint32_t (&out)[4]) {
+  raw_word<true>(w, out);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) out[i] = b2_as_u32(__hsub2(u32_as_b2(out[i]), u32_as_b2(bias)));
+}
+
+template <int kNTiles, bool kOffset, int kCW, bool kBf16 = false>
 __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
     const __grid_constant__ CUtensorMap tmap_z, const uint32_t* __restrict__ qweight,
-    const __half* __restrict__ X, int M, int64_t N, int64_t K, const float* __restrict__ inv_s,
-    __half* __restrict__ Y, G4Smem lay, unsigned flags) {
+    const act_t<kBf16>* __restrict__ X, int M, int64_t N, int64_t K,
+    const float* __restrict__ inv_s, act_t<kBf16>* __restrict__ Y, G4Smem lay, unsigned flags) {
   static_assert(kG4Groups % kCW == 0, "consumer warps must divide the unit's groups");
   constexpr int kGPW = kG4Groups / kCW;   // groups per consumer warp and unit
   constexpr int kTok = 8 * kNTiles;
   extern __shared__ __align__(128) uint8_t smem[];
-  __half* xs = reinterpret_cast<__half*>(smem);
+  act_t<kBf16>* xs = reinterpret_cast<act_t<kBf16>*>(smem);
   float* cc = reinterpret_cast<float*>(smem + lay.c_off());
   uint8_t* slots = smem + lay.slot_off();
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bar_off());
@@ -369,8 +394,9 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
   if (kOffset) {
     // One pass over X: x <- fp16(x * inv_s), columns k%8 in {2,3,6,7} divided by 16 (exact
     // in fp16), and per (group, token < M) C1 = 1024 * sum(xs) and C2 = sum(x) from the staged
-    // values; tokens >= M get zeros. 8 threads per (group, token) pair, 2 chunks of 8 each,
-    // 4 pairs per warp and pass, three xor-shuffles.
+    // values; tokens >= M get zeros. (bf16: x <- bf16(x * inv_s), no division, C2 = sum(x)
+    // and C1 = 128 * C2.) 8 threads per (group, token) pair, 2 chunks of 8 each, 4 pairs per
+    // warp and pass, three xor-shuffles.
     const int sub = lane & 7;
     const int npairs = G * M;
     const __half2 sixteenth = __float2half2_rn(0.0625f);
@@ -385,22 +411,19 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
         uint4 v = live ? src[h] : make_uint4(0u, 0u, 0u, 0u);
         if (inv_s != nullptr && live) {
           const int k = g * kGroup + 16 * sub + 8 * h;
-          const float4 s0 = *reinterpret_cast<const float4*>(inv_s + k);
-          const float4 s1 = *reinterpret_cast<const float4*>(inv_s + k + 4);
-          float2 f;
-          f = __half22float2(u32_as_h2(v.x)); v.x = h2_as_u32(__floats2half2_rn(f.x * s0.x, f.y * s0.y));
-          f = __half22float2(u32_as_h2(v.y)); v.y = h2_as_u32(__floats2half2_rn(f.x * s0.z, f.y * s0.w));
-          f = __half22float2(u32_as_h2(v.z)); v.z = h2_as_u32(__floats2half2_rn(f.x * s1.x, f.y * s1.y));
-          f = __half22float2(u32_as_h2(v.w)); v.w = h2_as_u32(__floats2half2_rn(f.x * s1.z, f.y * s1.w));
+          v = scale8<kBf16>(v, *reinterpret_cast<const float4*>(inv_s + k),
+                            *reinterpret_cast<const float4*>(inv_s + k + 4));
         }
-        v.y = h2_as_u32(__hmul2(u32_as_h2(v.y), sixteenth));
-        v.w = h2_as_u32(__hmul2(u32_as_h2(v.w), sixteenth));
+        if constexpr (!kBf16) {
+          v.y = h2_as_u32(__hmul2(u32_as_h2(v.y), sixteenth));
+          v.w = h2_as_u32(__hmul2(u32_as_h2(v.w), sixteenth));
+        }
         if (live) src[h] = v;
-        const float2 lx = __half22float2(u32_as_h2(v.x)), hy = __half22float2(u32_as_h2(v.y));
-        const float2 lz = __half22float2(u32_as_h2(v.z)), hw = __half22float2(u32_as_h2(v.w));
+        const float2 lx = act2_to_float2<kBf16>(v.x), hy = act2_to_float2<kBf16>(v.y);
+        const float2 lz = act2_to_float2<kBf16>(v.z), hw = act2_to_float2<kBf16>(v.w);
         const float lo = (lx.x + lx.y) + (lz.x + lz.y), hi = (hy.x + hy.y) + (hw.x + hw.y);
         c1 += lo + hi;
-        c2 += lo + 16.0f * hi;
+        c2 += kBf16 ? lo + hi : lo + 16.0f * hi;
       }
 #pragma unroll
       for (int o = 1; o < 8; o <<= 1) {
@@ -408,7 +431,7 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
         c2 += __shfl_xor_sync(0xffffffffu, c2, o);
       }
       if (sub == 0 && live) {
-        cc[(g * kTok + m) * 2] = 1024.0f * c1;
+        cc[(g * kTok + m) * 2] = kBf16 ? 128.0f * c2 : 1024.0f * c1;
         cc[(g * kTok + m) * 2 + 1] = c2;
       }
     }
@@ -416,19 +439,13 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
       if (i % kTok >= M) { cc[2 * i] = 0.0f; cc[2 * i + 1] = 0.0f; }
     named_bar_sync(1, kCW * 32);
   } else if (inv_s != nullptr) {
-    // x <- fp16(x * inv_s)
+    // x <- fp16(x * inv_s) (bf16 for bf16 activations)
     const int n8 = M * Ki / 8;
     for (int i = threadIdx.x; ok && i < n8; i += kCW * 32) {
-      uint4 v = reinterpret_cast<uint4*>(xs)[i];
       const int k = (i * 8) % Ki;
-      const float4 s0 = *reinterpret_cast<const float4*>(inv_s + k);
-      const float4 s1 = *reinterpret_cast<const float4*>(inv_s + k + 4);
-      float2 f;
-      f = __half22float2(u32_as_h2(v.x)); v.x = h2_as_u32(__floats2half2_rn(f.x * s0.x, f.y * s0.y));
-      f = __half22float2(u32_as_h2(v.y)); v.y = h2_as_u32(__floats2half2_rn(f.x * s0.z, f.y * s0.w));
-      f = __half22float2(u32_as_h2(v.z)); v.z = h2_as_u32(__floats2half2_rn(f.x * s1.x, f.y * s1.y));
-      f = __half22float2(u32_as_h2(v.w)); v.w = h2_as_u32(__floats2half2_rn(f.x * s1.z, f.y * s1.w));
-      reinterpret_cast<uint4*>(xs)[i] = v;
+      reinterpret_cast<uint4*>(xs)[i] =
+          scale8<kBf16>(reinterpret_cast<uint4*>(xs)[i], *reinterpret_cast<const float4*>(inv_s + k),
+                        *reinterpret_cast<const float4*>(inv_s + k + 4));
     }
     named_bar_sync(1, kCW * 32);
   }
@@ -483,18 +500,27 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
         const uint32_t wordsB[4] = {wB[q].x, wB[q].y, wB[q].z, wB[q].w};
         const int kx = g * kGroup + 32 * c;
         __half2 loA, hiA, loB, hiB;
+        uint32_t bA = 0, bB = 0;   // bf16 bias pairs (128 + z)
         if (!kOffset) {
-          loA = u32_as_h2((0x6400u | zAi[q]) * 0x00010001u);
-          hiA = u32_as_h2((0xD400u | (zAi[q] << 4)) * 0x00010001u);
-          loB = u32_as_h2((0x6400u | zBi[q]) * 0x00010001u);
-          hiB = u32_as_h2((0xD400u | (zBi[q] << 4)) * 0x00010001u);
+          if constexpr (kBf16) {
+            bA = (0x4300u | zAi[q]) * 0x00010001u;
+            bB = (0x4300u | zBi[q]) * 0x00010001u;
+          } else {
+            loA = u32_as_h2((0x6400u | zAi[q]) * 0x00010001u);
+            hiA = u32_as_h2((0xD400u | (zAi[q] << 4)) * 0x00010001u);
+            loB = u32_as_h2((0x6400u | zBi[q]) * 0x00010001u);
+            hiB = u32_as_h2((0xD400u | (zBi[q] << 4)) * 0x00010001u);
+          }
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t va[4], vb[4];
           if (kOffset) {
-            raw_word(wordsA[j], va);
-            raw_word(wordsB[j], vb);
+            raw_word<kBf16>(wordsA[j], va);
+            raw_word<kBf16>(wordsB[j], vb);
+          } else if constexpr (kBf16) {
+            dequant_word_qz_bf16(wordsA[j], bA, va);
+            dequant_word_qz_bf16(wordsB[j], bB, vb);
           } else {
             dequant_word_qz(wordsA[j], loA, hiA, va);
             dequant_word_qz(wordsB[j], loB, hiB, vb);
@@ -506,9 +532,9 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
             if (m < M && AWQ_IN_BOUNDS(kx + 8 * j + 8 <= Ki))
               xv = *reinterpret_cast<const uint4*>(xs + m * Ki + kx + 8 * j);
             const uint32_t a0[4] = {va[0], vb[0], va[1], vb[1]};
-            mma_16816(acc[t][j], a0, xv.x, xv.y);
+            mma_16816<kBf16>(acc[t][j], a0, xv.x, xv.y);
             const uint32_t a1[4] = {va[2], vb[2], va[3], vb[3]};
-            mma_16816(acc[t][j], a1, xv.z, xv.w);
+            mma_16816<kBf16>(acc[t][j], a1, xv.z, xv.w);
           }
         }
 #pragma unroll
@@ -555,12 +581,12 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
         const int64_t nA = tile * kGemvRows + r, nB = nA + 8;
         const int m0 = 8 * t + 2 * c, m1 = m0 + 1;
         if (nA < N && AWQ_IN_BOUNDS(tile < t1)) {
-          if (m0 < M) Y[static_cast<int64_t>(m0) * N + nA] = __float2half_rn(v[0]);
-          if (m1 < M) Y[static_cast<int64_t>(m1) * N + nA] = __float2half_rn(v[1]);
+          if (m0 < M) Y[static_cast<int64_t>(m0) * N + nA] = float_to_act<kBf16>(v[0]);
+          if (m1 < M) Y[static_cast<int64_t>(m1) * N + nA] = float_to_act<kBf16>(v[1]);
         }
         if (nB < N && AWQ_IN_BOUNDS(tile < t1)) {
-          if (m0 < M) Y[static_cast<int64_t>(m0) * N + nB] = __float2half_rn(v[2]);
-          if (m1 < M) Y[static_cast<int64_t>(m1) * N + nB] = __float2half_rn(v[3]);
+          if (m0 < M) Y[static_cast<int64_t>(m0) * N + nB] = float_to_act<kBf16>(v[2]);
+          if (m1 < M) Y[static_cast<int64_t>(m1) * N + nB] = float_to_act<kBf16>(v[3]);
         }
       }
       named_bar_sync(1, kCW * 32);

@@ -166,10 +166,13 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
     zeros[j * N + nb + t - 32] = sh_zero[t - 32];
 }
 
-// Search operand: for grid point a, E[a][n][k] = fp16(deq[n,k] * inv_a[k] - w[n,k]) with
+// Search operand: for grid point a, e = deq[n,k] * inv_a[k] - w[n,k] in fp32, with
 // deq = (q - z) * sc from the quantizer above and inv_a = 1 / s_a (correctly rounded, from
-// a table); rows N..N_pad-1 are written as zeros so that 128-row tiles never straddle two
-// grid points.
+// a table), stored in two fp16 parts, hi = fp16(e) and lo = fp16((e - hi) * 2^12) (e - hi
+// is exact in fp32, the scaling by a power of 2 too): hi + 2^-12 lo represents e to about 22
+// significant bits instead of fp16's 11. Row n of grid point a is row a * N_pad + n of a
+// [rows, 2K] matrix holding hi in columns 0..K-1 and lo in K..2K-1; rows N..N_pad-1 are
+// written as zeros so that 128-row tiles never straddle two grid points.
 template <int kBits>
 __global__ void __launch_bounds__(256) search_build_error_kernel(
     const __half* __restrict__ W, int64_t N, int64_t K, int64_t N_pad,
@@ -189,6 +192,7 @@ __global__ void __launch_bounds__(256) search_build_error_kernel(
   const QuantGroup g = group_params<kBits>(w);
   if (n >= N_pad) return;
   uint4 out[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+  uint4 out_lo[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
   if (valid) {
     const float4* ip = reinterpret_cast<const float4*>(inv_table + a * K + k0);
     float inv[16];
@@ -197,7 +201,7 @@ __global__ void __launch_bounds__(256) search_build_error_kernel(
       const float4 v = ip[qd];
       inv[4 * qd] = v.x; inv[4 * qd + 1] = v.y; inv[4 * qd + 2] = v.z; inv[4 * qd + 3] = v.w;
     }
-    uint32_t e2[8];
+    uint32_t e2[8], l2[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       float e[2];
@@ -208,15 +212,25 @@ __global__ void __launch_bounds__(256) search_build_error_kernel(
         const float deq = __fmul_rn(__fsub_rn(q, g.z), g.sc);
         e[u] = __fsub_rn(__fmul_rn(deq, inv[idx]), w_raw[idx]);
       }
-      e2[i] = h2_as_u32(__floats2half2_rn(e[0], e[1]));
+      const __half2 hi = __floats2half2_rn(e[0], e[1]);
+      const float2 hf = __half22float2(hi);
+      e2[i] = h2_as_u32(hi);
+      l2[i] = h2_as_u32(__floats2half2_rn(__fmul_rn(__fsub_rn(e[0], hf.x), 4096.0f),
+                                          __fmul_rn(__fsub_rn(e[1], hf.y), 4096.0f)));
     }
     out[0] = make_uint4(e2[0], e2[1], e2[2], e2[3]);
     out[1] = make_uint4(e2[4], e2[5], e2[6], e2[7]);
+    out_lo[0] = make_uint4(l2[0], l2[1], l2[2], l2[3]);
+    out_lo[1] = make_uint4(l2[4], l2[5], l2[6], l2[7]);
   }
   if (!AWQ_IN_BOUNDS(a < gridDim.z && k0 + 16 <= K)) return;
-  uint4* dst = reinterpret_cast<uint4*>(E + a * N_pad * K + n * K + k0);
+  __half* row = E + (a * N_pad + n) * (2 * K);
+  uint4* dst = reinterpret_cast<uint4*>(row + k0);
   dst[0] = out[0];
   dst[1] = out[1];
+  uint4* dst_lo = reinterpret_cast<uint4*>(row + K + k0);
+  dst_lo[0] = out_lo[0];
+  dst_lo[1] = out_lo[1];
 }
 
 // inv_table[a][k] = 1 / s_table[a][k], correctly rounded.
