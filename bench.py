@@ -192,26 +192,28 @@ class ClockSampler:
 class DecodeShape:
     """One decode shape's rotating weight copies and its input/output buffers."""
 
-    def __init__(self, awq, N, K, m_max, l2_bytes, device):
+    def __init__(self, awq, N, K, m_max, l2_bytes, device, bf16=False, bits=4):
         W, mag, X = synth.decode_layer(N, K, m_max)
         s = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(device)
         Wd = torch.from_numpy(W).to(device)
-        base = awq.awq_quantize_pack(Wd, s, 4)
+        self.bits = bits
+        base = awq.awq_quantize_pack(Wd, s, bits)
         del Wd
         per_copy = sum(t.numel() * t.element_size() for t in base)
         self.copies = max(2, math.ceil(2 * l2_bytes / per_copy))
         self.w = [base] + [tuple(t.clone() for t in base) for _ in range(self.copies - 1)]
         self.N, self.K = N, K
-        self.X = torch.from_numpy(X).to(device)
-        self.Y = torch.empty(m_max, N, dtype=torch.float16, device=device)
-        self.Xh = torch.from_numpy(X).pin_memory()
-        self.Yh = torch.empty(m_max, N, dtype=torch.float16).pin_memory()
+        dt = torch.bfloat16 if bf16 else torch.float16
+        self.X = torch.from_numpy(X).to(device).to(dt)
+        self.Y = torch.empty(m_max, N, dtype=dt, device=device)
+        self.Xh = torch.from_numpy(X).to(dt).pin_memory()
+        self.Yh = torch.empty(m_max, N, dtype=dt).pin_memory()
 
     def call(self, awq, M, r, stream=None):
         # the packed weights are static (no kernel writes them between steps), which is the
         # AWQ_GEMM_WEIGHTS_READY contract: each GEMM may stream them while the previous runs
         qw, sc, z = self.w[r % self.copies]
-        awq.awq_gemm_w4a16(self.X[:M], qw, sc, z, self.N, self.K, 4, out=self.Y[:M],
+        awq.awq_gemm_w4a16(self.X[:M], qw, sc, z, self.N, self.K, self.bits, out=self.Y[:M],
                            stream=stream, weights_ready=True)
 
 
@@ -307,17 +309,28 @@ def time_call(fn, reps, warm=1):
 
 def decoder_layer_rows(awq, dev, pk):
     """The other hot-path rows on the 7B-shaped decoder layer and its 65536-token calibration
-    batch: activation statistics, the 20-point searches (q/k/v and gate/up jointly), packing,
-    and the W4A16 GEMM of every linear over the calibration batch -- timed per stage and as
-    one pipeline. Also quantize-and-pack on the largest prefill weight."""
+    batch: activation statistics, down_proj's calibration input computed as the gated MLP
+    produces it (silu(X W_gate^T) * (X W_up^T) from the fp16 weights), the 20-point searches
+    (q/k/v and gate/up jointly), packing, and the W4A16 GEMM of every linear over the
+    calibration batch -- timed per stage and as one pipeline. Also quantize-and-pack on the
+    largest prefill weight."""
     rows = {}
-    acts = synth.decoder_layer_activations()
+    acts = synth.decoder_layer_activations(names=("hidden", "o_in"))
     Ws = synth.decoder_layer_weights()
     alphas = torch.from_numpy(np.arange(20, dtype=np.float32) / np.float32(20)).to(dev)
     Xd = {k: torch.from_numpy(v).to(dev) for k, v in acts.items()}
     del acts
     Wd = {k: torch.from_numpy(v).to(dev) for k, v in Ws.items()}
     del Ws
+    # down_proj's calibration input: the gated MLP's output on the hidden state
+    Mtok = int(Xd["hidden"].shape[0])
+    Xd["down_in"] = torch.empty(Mtok, Wd["gate_proj"].shape[0], dtype=torch.float16, device=dev)
+    t = time_call(lambda: awq.awq_silu_mul_gemm(Xd["hidden"], Wd["gate_proj"], Wd["up_proj"],
+                                                out=Xd["down_in"]), 3)
+    fl = 4 * Mtok * Wd["gate_proj"].shape[0] * Wd["gate_proj"].shape[1]
+    rows["gated_mlp_input"] = {"M": Mtok, "I": Wd["gate_proj"].shape[0],
+                               "K": Wd["gate_proj"].shape[1], "ms": t * 1e3,
+                               "TFLOP/s": fl / t / 1e12, "frac_tensor": fl / t / 1e12 / pk["bf16_tflops"]}
 
     # act_stats (HBM-bound: 2MK bytes)
     out = []
@@ -342,15 +355,17 @@ def decoder_layer_rows(awq, dev, pk):
                      device=dev)
     t = time_call(lambda: awq.awq_search_scale(Wgu, X, sx, alphas, 4, workspace=ws), 2)
     flops = 20 * 2 * M * Ngu * K
+    # the error operand's two fp16 parts each go through the tensor cores: 2x the MMA work
     rows["search_gate_up"] = {"M": M, "N": Ngu, "K": K, "grid": 20, "ms": t * 1e3,
-                              "TFLOP/s": flops / t / 1e12,
-                              "frac_tensor": flops / t / 1e12 / pk["bf16_tflops"]}
+                              "TFLOP/s (algorithmic 20*2MNK)": flops / t / 1e12,
+                              "TFLOP/s (executed, two-part operand)": 2 * flops / t / 1e12,
+                              "frac_tensor_executed": 2 * flops / t / 1e12 / pk["bf16_tflops"]}
     del ws, Wgu
     torch.cuda.empty_cache()
 
-    # the whole layer as one pipeline: stats -> 4 searches -> 7 packs -> 7 GEMMs over the batch
-    # (outputs and workspaces allocated before the timed region)
-    Mtok = int(Xd["hidden"].shape[0])
+    # the whole layer as one pipeline: stats -> gated-MLP input of down_proj and its stats ->
+    # 4 searches -> 7 packs -> 7 GEMMs over the batch (outputs and workspaces allocated before
+    # the timed region)
     y_buf = torch.empty(Mtok * max(W.shape[0] for W in Wd.values()), dtype=torch.float16,
                         device=dev)
     g_ws = torch.empty(awq.lib().awq_gemm_workspace_size(Mtok, 1, max(W.shape[1] for W in
@@ -369,6 +384,7 @@ def decoder_layer_rows(awq, dev, pk):
     search_ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
     ev[0].record()
+    awq.awq_silu_mul_gemm(Xd["hidden"], Wd["gate_proj"], Wd["up_proj"], out=Xd["down_in"])
     stats = {name: awq.awq_act_stats(Xd[name]) for name in ("hidden", "o_in", "down_in")}
     ev[1].record()
     for xname, names in jobs:
@@ -398,7 +414,7 @@ def decoder_layer_rows(awq, dev, pk):
     st_gemm_only = ev3b.elapsed_time(ev[4]) / 1e3
     rows["decoder_layer_pipeline"] = {
         "tokens": int(Xd["hidden"].shape[0]), "seconds": sum(st),
-        "act_stats_s": st[0], "search_s": st[1], "pack_s": st[2], "gemm_s": st[3],
+        "stats_and_gated_input_s": st[0], "search_s": st[1], "pack_s": st[2], "gemm_s": st[3],
         "search_TFLOP/s": search_flops / st[1] / 1e12,
         "gemm_TFLOP/s": gemm_flops / st_gemm_only / 1e12,
         "alpha_index": {n: int(chosen[n][0].item()) for n in chosen},
@@ -590,7 +606,7 @@ def run_b200(args, world, rank, local):
     # ---- prefill at M = 2048 (4-bit on the three shapes, then the 3-bit variant)
     prefill = []
     pf_cases = [(N, K, 4) for (N, K) in synth.PREFILL_SHAPES] + [(*synth.PREFILL_SHAPES[0], 3)]
-    for (N, K, bits) in (pf_cases if args.only not in ("decode", "batched") else []):
+    for (N, K, bits) in (pf_cases if args.only in ("all", "prefill") else []):
         m_list = synth.PREFILL_M if bits == 4 else [2048]
         W, mag, X = synth.prefill_layer(N, K, max(m_list))
         s = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(dev)
@@ -618,6 +634,45 @@ def run_b200(args, world, rank, local):
     pf_flops = sum(2 * 2048 * p["N"] * p["K"] for p in pf4)
     pf_time = sum(p["ms"] for p in pf4) / 1e3
     pf_value = pf_flops / pf_time / 1e12 if pf4 else None
+
+    # ---- bf16 activations: the headline decode step and the M = 2048 prefill GEMM
+    bf16 = {}
+    if args.only in ("all", "bf16"):
+        shapes_b = [DecodeShape(awq, N, K, 1, l2, dev, bf16=True) for (N, K) in synth.DECODE_SHAPES]
+        for sh in shapes_b:
+            sh.call(awq, 1, 0)
+        t = time_steps(lambda r: [sh.call(awq, 1, r) for sh in shapes_b], 200, 10, stream, world)
+        b = sum(gemm_bytes(1, sh.N, sh.K) for sh in shapes_b)
+        bf16["decode_M1_step"] = {"us_per_step": t / 200 * 1e6, "GB/s": b * 200 / t / 1e9,
+                                  "frac_hbm": b * 200 / t / 1e9 / pk["hbm_gbs"]}
+        del shapes_b
+        # 3-bit codes, fp16 activations: the same headline step
+        shapes_3 = [DecodeShape(awq, N, K, 1, l2, dev, bits=3) for (N, K) in synth.DECODE_SHAPES]
+        for sh in shapes_3:
+            sh.call(awq, 1, 0)
+        t = time_steps(lambda r: [sh.call(awq, 1, r) for sh in shapes_3], 200, 10, stream, world)
+        b = sum(gemm_bytes(1, sh.N, sh.K, 3) for sh in shapes_3)
+        bf16["decode_M1_step_3bit_fp16"] = {"us_per_step": t / 200 * 1e6,
+                                            "GB/s": b * 200 / t / 1e9,
+                                            "frac_hbm": b * 200 / t / 1e9 / pk["hbm_gbs"]}
+        del shapes_3
+        N, K = synth.PREFILL_SHAPES[0]
+        W, mag, X = synth.prefill_layer(N, K, 2048)
+        s_ = torch.from_numpy(np.power(mag.astype(np.float64), 0.5).astype(np.float32)).to(dev)
+        Wt = torch.from_numpy(W).to(dev)
+        del W
+        packs = [awq.awq_quantize_pack(Wt, s_, 4)]
+        del Wt
+        packs.append(tuple(t_.clone() for t_ in packs[0]))
+        Xb = torch.from_numpy(X).to(dev).to(torch.bfloat16)
+        Yb = torch.empty(2048, N, dtype=torch.bfloat16, device=dev)
+        t = time_steps(lambda r: awq.awq_gemm_w4a16(Xb, *packs[r % 2], N, K, 4, out=Yb), 20, 3,
+                       stream, world)
+        tfl = 2 * 2048 * N * K * 20 / t / 1e12
+        bf16["prefill_M2048_28672x8192"] = {"ms": t / 20 * 1e3, "TFLOP/s": tfl,
+                                            "frac_tensor": tfl / pk["bf16_tflops"]}
+        del packs, Xb, Yb
+        torch.cuda.empty_cache()
 
     rows = decoder_layer_rows(awq, dev, pk) if args.only == "all" else None
 
@@ -658,6 +713,7 @@ def run_b200(args, world, rank, local):
                     "kernel": "tc_gemm_kernel"},
         "sweep": sweep,
         "batched": batched,
+        "bf16_and_3bit": bf16,
         "rows": rows,
         "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": cpu_cores,
                          "kind": "oracle", "sample": cpu_desc, "seconds": cpu_t},
@@ -674,7 +730,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--only", choices=["all", "decode", "batched", "prefill", "rows", "profile"],
+    ap.add_argument("--only", choices=["all", "decode", "batched", "prefill", "bf16", "rows",
+                                       "profile"],
                     default="all",
                     help="run one section only (used by the profiling commands)")
     args = ap.parse_args()

@@ -189,8 +189,9 @@ AWQ_API awq_status awq_silu_mul_gemm(const awq_f16* X, int64_t M, const awq_f16*
  * decode kernels apply inv_s to the activations in fp32 (x' = fp16(x * inv_s)); the
  * tensor-core kernel folds it into the dequantized weights (fp16(scale * inv_s[k]) per k),
  * so no extra pass over X is made.
- * M <= 16 with 4 bits runs a decode kernel (HBM-bound GEMV; for 8 < M <= 16 only when X
- * fits in one CTA's shared memory); other calls (and 3 bits) run the tensor-core kernel.
+ * M <= 16 runs a decode kernel (HBM-bound GEMV, 4 or 3 bits; when N is a multiple of 16 and
+ * X fits in one CTA's shared memory, or, for fp16 4-bit M <= 8, a register-streaming kernel);
+ * other calls run the tensor-core kernel.
  * X: fp16 [M, K]; Y: fp16 [M, N]. M = 0 or N = 0 is a no-op.
  * flags: 0, or AWQ_GEMM_WEIGHTS_READY. The kernels are launched with programmatic dependent
  * launch, so a kernel of this call may start while the kernel launched just before it on

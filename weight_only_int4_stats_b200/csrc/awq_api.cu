@@ -98,15 +98,17 @@ awq_status launch_tc(const void* Xop, int64_t M, const void* Aop, int64_t a_rows
     attr_set[dev].store(true, std::memory_order_release);
   }
   CUtensorMap tx, ta;
+  // B operand rows M x (K, or 2K for the two-part normalised Gram matrix) columns
   if (!make_tmap_2d(&tx, Xop, kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                    2, M, args.K, BN, awq::kTcBK, true))
+                    2, M, kA == ASrc::kGram ? 2 * args.K : args.K, BN, awq::kTcBK, true))
     return AWQ_ERR_CUDA;
-  if (kA == ASrc::kSplit16) {   // [a_rows, 2K]: the hi part, then the lo part, of each row
+  if (kA == ASrc::kSplit16 || kA == ASrc::kGram) {   // [a_rows, 2K]: hi part, then lo part
     if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a_rows, 2 * args.K,
                       awq::kTcBM, awq::kTcBK, true))
       return AWQ_ERR_CUDA;
-  } else if (kA == ASrc::kPair16) {   // two [a_rows, K] weights; the second map goes in ts
+  } else if (kA == ASrc::kPair16 || kA == ASrc::kFp16x1) {   // [a_rows, K] fp16 (kPair16:
+                                                                  // the second map goes in ts)
     if (!make_tmap_2d(&ta, Aop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a_rows, args.K, awq::kTcBM,
                       awq::kTcBK, true))
       return AWQ_ERR_CUDA;
@@ -143,7 +145,10 @@ awq_status launch_tc(const void* Xop, int64_t M, const void* Aop, int64_t a_rows
   if (a.k_splits < 1) a.k_splits = 1;
   const int64_t units = static_cast<int64_t>(a.m_tiles) * a.row_tiles * a.k_splits;
   const int64_t sms = num_sms();
-  const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);   // persistent
+  // persistent, one CTA per SM; the fp32-store epilogue instead takes one CTA per output tile,
+  // so that a tile's contraction slices are consecutive units of the same CTA
+  const int64_t want = kEpi == Epi::kStoreF32 ? units / a.k_splits : sms;
+  const unsigned grid = static_cast<unsigned>(units < want ? units : want);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(awq::kTcThreads);
@@ -167,118 +172,115 @@ awq_status launch_tc_bn(const void* Xop, int64_t M, const void* Aop, int64_t a_r
   return launch_tc<256, kA, kEpi, kBf16>(Xop, M, Aop, a_rows, args, st, Aop2);
 }
 
-// Streaming decode GEMM (M <= 16, 4-bit), launched with programmatic dependent launch.
+// Streaming decode GEMM (M <= 16), launched with programmatic dependent launch.
 constexpr int kSmemLimit = 232448;   // 227 KB per CTA on sm_100
-// Two CTAs share an SM's 228 KB when each stays within this (1 KB per CTA is reserved).
-constexpr int kCoResidentSmem = (233472 - 2 * 1024) / 2;
-
 static_assert(awq::kGemvWeightsReady == AWQ_GEMM_WEIGHTS_READY, "flag values must agree");
 static_assert((AWQ_GEMM_WEIGHTS_READY & AWQ_GEMM_BF16) == 0, "flags are distinct bits");
 
-struct GemvConfig {
-  int cw;       // consumer warps (8 or 16)
-  int slots;    // ring depth
-  int per_sm;   // CTAs of this grid per SM
-  int smem;     // dynamic shared memory per CTA
-  awq::G4Smem lay;
-};
+// Two CTAs of the streaming kernel fit on one SM when each takes at most half of its 228 KB
+// (less 1 KB reserved per CTA): the next launch's CTAs then start beside this one's.
+constexpr int kCoResidentSmem = (233472 - 2 * 1024) / 2;
 
-// The launch shape of the streaming decode kernel: 8 consumer warps, one CTA per SM and the
-// deepest ring (up to kGSMaxSlots) that leaves room for the next launch's CTA on the same SM;
-// when X is too large for that, the deepest ring within one CTA's shared memory. Returns
-// false when the shape does not suit the kernel: N not in whole 16-row tiles, or X plus a
-// two-slot ring beyond one CTA's shared memory (kNTiles = 1 for M <= 8, 2 for M <= 16).
-bool gemv_config(int64_t M, int64_t N, int64_t K, int cw, int slots_max, int per_sm,
-                 GemvConfig* out) {
+// The streaming kernel's shared-memory plan for a shape: the deepest ring (6 down to 2 slots)
+// that leaves room for a co-resident CTA, else the deepest that fits one CTA.
+bool gemv_config(int64_t M, int64_t N, int64_t K, awq::G4Smem* out) {
   if (M < 1 || M > 16 || N % 16 != 0 || K / awq::kGroup > 65535) return false;
-  if (M * K * 2 > kSmemLimit) return false;
   const int nt = M <= 8 ? 1 : 2;
-  for (int budget : {kCoResidentSmem, kSmemLimit}) {
-    for (int slots = slots_max; slots >= 2; --slots) {
-      const awq::G4Smem l = awq::G4Smem::make(static_cast<int>(M), K, nt, slots, cw);
+  for (int budget : {kCoResidentSmem, kSmemLimit})
+    for (int slots = awq::kGSMaxSlots; slots >= 2; --slots) {
+      const awq::G4Smem l = awq::G4Smem::make(static_cast<int>(M), K, nt, slots);
       if (l.total(nt) <= budget) {
-        *out = GemvConfig{cw, slots, per_sm, l.total(nt), l};
+        *out = l;
         return true;
       }
     }
-  }
   return false;
 }
 
+// Whether the streaming decode kernel takes this shape: N in whole 16-row tiles and X (plus the
+// small sums, the reduction buffer and a two-slot ring) within one CTA's shared memory.
 bool gemv_stream_fits(int64_t M, int64_t N, int64_t K) {
-  GemvConfig c;
-  return gemv_config(M, N, K, 8, awq::kGSMaxSlots, 1, &c);
+  awq::G4Smem l;
+  return gemv_config(M, N, K, &l);
 }
 
-template <int kNTiles, bool kOffset, int kCW, bool kBf16 = false>
-awq_status launch_gemv_stream_cfg(const GemvConfig& cfgv, const void* x, int64_t M,
-                                  const uint32_t* qweight, const __half* scales,
-                                  const uint8_t* zeros, int64_t N, int64_t K, const float* inv_s,
-                                  unsigned flags, void* y, cudaStream_t st) {
+template <int kNTiles, bool kOffset, bool kBf16, int kBits>
+awq_status launch_gemv_stream_t(const void* x, int64_t M, const uint32_t* qweight,
+                                const __half* scales, const uint8_t* zeros, int64_t N, int64_t K,
+                                const float* inv_s, unsigned flags, void* y, cudaStream_t st) {
   using A = awq::act_t<kBf16>;
   static std::atomic<bool> attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
-  auto kern = awq::gemv_stream_kernel<kNTiles, kOffset, kCW, kBf16>;
+  auto kern = awq::gemv_stream_kernel<kNTiles, kOffset, kBf16, kBits>;
   if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
         cudaSuccess)
       return AWQ_ERR_CUDA;
     attr_set[dev].store(true, std::memory_order_release);
   }
-  const int64_t tiles = N / 16;
-  const int64_t resident = static_cast<int64_t>(num_sms()) * cfgv.per_sm;
-  const unsigned grid = static_cast<unsigned>(tiles < resident ? tiles : resident);
+  awq::G4Smem lay;
+  if (!gemv_config(M, N, K, &lay)) return AWQ_ERR_UNSUPPORTED;
+  // packed codes [N, K * bits / 32] words in boxes of 16 rows x 32 words (128 B, swizzled);
+  // scales [G, N] fp16 and zero points [G, N] uint8 in boxes of 16 groups x 16 rows
   CUtensorMap tw, ts, tz;
-  if (!make_tmap_2d(&tw, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, 16,
-                    awq::kG4KC / 8, false) ||
+  if (!make_tmap_2d(&tw, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K * kBits / 32,
+                    awq::kGemvRows, 32, true) ||
       !make_tmap_2d(&ts, scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K / awq::kGroup, N,
-                    awq::kG4Groups, 16, false) ||
+                    awq::kG4Groups, awq::kGemvRows, false) ||
       !make_tmap_2d(&tz, zeros, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / awq::kGroup, N,
-                    awq::kG4Groups, 16, false))
+                    awq::kG4Groups, awq::kGemvRows, false))
     return AWQ_ERR_CUDA;
+  const int64_t tiles = N / awq::kGemvRows;
+  const int64_t sms = num_sms();
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3((kCW + 1) * 32);
-  cfg.dynamicSmemBytes = static_cast<size_t>(cfgv.smem);
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles < sms ? tiles : sms));   // one CTA per SM
+  cfg.blockDim = dim3(awq::kG4Threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(lay.total(kNTiles));
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const int m32 = static_cast<int>(M);
-  if (cudaLaunchKernelEx(&cfg, kern, tw, ts, tz, qweight, static_cast<const A*>(x), m32, N, K,
-                         inv_s, static_cast<A*>(y), cfgv.lay, flags) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kern, tw, ts, tz, qweight, static_cast<const A*>(x),
+                         static_cast<int>(M), N, K, inv_s, static_cast<A*>(y), lay,
+                         flags) != cudaSuccess)
     return AWQ_ERR_CUDA;
   return launch_status();
 }
 
+template <bool kBf16, int kBits>
+awq_status launch_gemv_stream_m(const void* x, int64_t M, const uint32_t* qweight,
+                                const __half* scales, const uint8_t* zeros, int64_t N, int64_t K,
+                                const float* inv_s, unsigned flags, void* y, cudaStream_t st) {
+  if (M == 1)
+    return launch_gemv_stream_t<1, true, kBf16, kBits>(x, M, qweight, scales, zeros, N, K, inv_s,
+                                                       flags, y, st);
+  if (M <= 8)
+    return launch_gemv_stream_t<1, false, kBf16, kBits>(x, M, qweight, scales, zeros, N, K,
+                                                        inv_s, flags, y, st);
+  return launch_gemv_stream_t<2, false, kBf16, kBits>(x, M, qweight, scales, zeros, N, K, inv_s,
+                                                      flags, y, st);
+}
+
 // Returns AWQ_ERR_UNSUPPORTED when the shape does not suit the streaming kernel; the caller
-// then uses the register-streaming kernel (M <= 8) or the tensor-core path.
+// then uses the register-streaming kernel (fp16, 4-bit, M <= 8) or the tensor-core path.
 awq_status launch_gemv_stream(const void* x, int64_t M, const uint32_t* qweight,
                               const __half* scales, const uint8_t* zeros, int64_t N, int64_t K,
-                              const float* inv_s, unsigned flags, void* y, cudaStream_t st) {
-  GemvConfig c;
-  if (!gemv_config(M, N, K, 8, awq::kGSMaxSlots, 1, &c)) return AWQ_ERR_UNSUPPORTED;
-  if (flags & AWQ_GEMM_BF16) {
-    if (M == 1)
-      return launch_gemv_stream_cfg<1, true, 8, true>(c, x, M, qweight, scales, zeros, N, K,
-                                                      inv_s, flags, y, st);
-    if (M <= 8)
-      return launch_gemv_stream_cfg<1, false, 8, true>(c, x, M, qweight, scales, zeros, N, K,
-                                                       inv_s, flags, y, st);
-    return launch_gemv_stream_cfg<2, false, 8, true>(c, x, M, qweight, scales, zeros, N, K,
-                                                     inv_s, flags, y, st);
-  }
-  if (M == 1)
-    return launch_gemv_stream_cfg<1, true, 8>(c, x, M, qweight, scales, zeros, N, K, inv_s,
-                                              flags, y, st);
-  if (M <= 8)
-    return launch_gemv_stream_cfg<1, false, 8>(c, x, M, qweight, scales, zeros, N, K, inv_s,
-                                               flags, y, st);
-  return launch_gemv_stream_cfg<2, false, 8>(c, x, M, qweight, scales, zeros, N, K, inv_s,
-                                             flags, y, st);
+                              int bits, const float* inv_s, unsigned flags, void* y,
+                              cudaStream_t st) {
+  if (!gemv_stream_fits(M, N, K)) return AWQ_ERR_UNSUPPORTED;
+  const bool bf16 = (flags & AWQ_GEMM_BF16) != 0;
+  if (bits == 3)
+    return bf16 ? launch_gemv_stream_m<true, 3>(x, M, qweight, scales, zeros, N, K, inv_s, flags,
+                                                y, st)
+                : launch_gemv_stream_m<false, 3>(x, M, qweight, scales, zeros, N, K, inv_s, flags,
+                                                 y, st);
+  return bf16 ? launch_gemv_stream_m<true, 4>(x, M, qweight, scales, zeros, N, K, inv_s, flags, y,
+                                              st)
+              : launch_gemv_stream_m<false, 4>(x, M, qweight, scales, zeros, N, K, inv_s, flags,
+                                               y, st);
 }
 
 int tc_bn_for(int64_t M) { return M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
@@ -485,26 +487,46 @@ namespace {
 // workspace stays bounded whatever the layer: at most this many bytes of E per chunk (at
 // least one grid point per chunk).
 constexpr size_t kSearchChunkBytes = size_t{1} << 30;
+// Column tile of the Gram-form loss GEMM (its N side is channels).
+constexpr int kGramBN = 128;
+
+// The loss is evaluated in its Gram form e G e^T (G = X^T X, N K^2 per grid point plus K^2 M
+// once) when that is cheaper than the direct ||E X^T||^2 (N K M per grid point) with margin:
+// the Gram MMAs cost 1.5 times the direct ones per product (three instead of two), so when
+// M >= 2K.
+bool search_uses_gram(int64_t M, int64_t K) { return M >= 2 * K; }
 
 struct SearchWs {
   int chunk;   // grid points per chunk
-  size_t table, inv, err, part, rows, total;
+  bool gram;
+  int64_t M_pad;
+  size_t table, inv, err, part, rows, xt, g, g2, rms, total;
 };
 SearchWs search_ws_layout(int64_t M, int64_t N, int64_t K, int n_alpha) {
   const int64_t N_pad = round_up(N, awq::kTcBM);
-  const int64_t m_tiles = (M + tc_bn_for(M) - 1) / tc_bn_for(M);
+  SearchWs w;
+  w.gram = search_uses_gram(M, K);
+  w.M_pad = round_up(M, awq::kGroup);
+  const int64_t m_tiles = w.gram ? K / kGramBN : (M + tc_bn_for(M) - 1) / tc_bn_for(M);
   const size_t per_point = static_cast<size_t>(N_pad) * 2 * K * sizeof(__half);   // hi, lo
   int64_t chunk = static_cast<int64_t>(kSearchChunkBytes / per_point);
   if (chunk < 1) chunk = 1;
   if (chunk > n_alpha) chunk = n_alpha;
-  SearchWs w;
   w.chunk = static_cast<int>(chunk);
   w.table = 0;
   w.inv = align256(static_cast<size_t>(n_alpha) * K * sizeof(float));
   w.err = w.inv + align256(static_cast<size_t>(n_alpha) * K * sizeof(float));
   w.part = w.err + align256(static_cast<size_t>(chunk) * per_point);
   w.rows = w.part + align256(static_cast<size_t>(chunk) * N_pad * m_tiles * sizeof(double));
-  w.total = w.rows + align256(static_cast<size_t>(n_alpha) * N * sizeof(double));
+  w.xt = w.rows + align256(static_cast<size_t>(n_alpha) * N * sizeof(double));
+  size_t end = w.xt;
+  if (w.gram) {   // X^T [K, M_pad] fp16, G [K, K] fp32, G' [K, 2K] fp16 parts, rms [K]
+    w.g = w.xt + align256(static_cast<size_t>(K) * w.M_pad * sizeof(__half));
+    w.g2 = w.g + align256(static_cast<size_t>(K) * K * sizeof(float));
+    w.rms = w.g2 + align256(static_cast<size_t>(K) * 2 * K * sizeof(__half));
+    end = w.rms + align256(static_cast<size_t>(K) * sizeof(float));
+  }
+  w.total = end;
   return w;
 }
 }  // namespace
@@ -536,14 +558,14 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
   if (N_pad / awq::kTcBM > 65535 || K / awq::kGroup > 65535) return AWQ_ERR_INVALID_ARG;
   const SearchWs lay = search_ws_layout(M, N, K, n_alpha);
   if (static_cast<int64_t>(lay.chunk) * N_pad / awq::kTcBM > 65535) return AWQ_ERR_INVALID_ARG;
+  if (lay.gram && (K / 32 > 65535 || lay.M_pad / 32 > 2147483647LL)) return AWQ_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < lay.total || !aligned16(workspace)) return AWQ_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* table = reinterpret_cast<float*>(ws + lay.table);
   __half* E = reinterpret_cast<__half*>(ws + lay.err);
   double* part = reinterpret_cast<double*>(ws + lay.part);
-  const int bn = tc_bn_for(M);
-  const int m_tiles = static_cast<int>((M + bn - 1) / bn);
+  const __half* x = reinterpret_cast<const __half*>(X);
   awq_status s;
 
   const float* S = s_table;
@@ -559,6 +581,37 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
     awq::inv_table_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(S, total, inv);
     if ((s = launch_status()) != AWQ_OK) return s;
   }
+  // Gram form: X^T (tokens contiguous, padded to whole groups), G = X^T X on the tensor
+  // cores, the channels' root mean squares, and G normalised to two fp16 parts
+  float* rms = nullptr;
+  const __half* G2 = nullptr;
+  if (lay.gram) {
+    __half* XT = reinterpret_cast<__half*>(ws + lay.xt);
+    float* G = reinterpret_cast<float*>(ws + lay.g);
+    __half* G2w = reinterpret_cast<__half*>(ws + lay.g2);
+    rms = reinterpret_cast<float*>(ws + lay.rms);
+    dim3 gt(static_cast<unsigned>(lay.M_pad / 32), static_cast<unsigned>((K + 31) / 32));
+    awq::transpose_pad_kernel<<<gt, 256, 0, st>>>(x, M, K, lay.M_pad, XT);
+    if ((s = launch_status()) != AWQ_OK) return s;
+    awq::TcArgs ga{};
+    ga.M = K;            // B rows: channels j
+    ga.N = K;
+    ga.N_pad = K;
+    ga.K = lay.M_pad;    // the contraction runs over tokens
+    ga.G = G;
+    // the contraction over tokens in slices of about 2048 (128 accumulation steps each)
+    ga.k_splits = static_cast<int>(lay.M_pad / 2048 > 1 ? lay.M_pad / 2048 : 1);
+    s = launch_tc<256, ASrc::kFp16x1, Epi::kStoreF32>(XT, K, XT, K, ga, st);
+    if (s != AWQ_OK) return s;
+    awq::gram_rms_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(G, K, M, rms);
+    if ((s = launch_status()) != AWQ_OK) return s;
+    dim3 gn(static_cast<unsigned>((K + 255) / 256), static_cast<unsigned>(K));
+    awq::gram_normalize_kernel<<<gn, 256, 0, st>>>(G, K, G2w);
+    if ((s = launch_status()) != AWQ_OK) return s;
+    G2 = G2w;
+  }
+  const int bn = lay.gram ? kGramBN : tc_bn_for(M);
+  const int m_tiles = lay.gram ? static_cast<int>(K / kGramBN) : static_cast<int>((M + bn - 1) / bn);
   double* rl = row_losses != nullptr ? row_losses : reinterpret_cast<double*>(ws + lay.rows);
   const __half* w = reinterpret_cast<const __half*>(W);
   for (int a0 = 0; a0 < n_alpha; a0 += lay.chunk) {
@@ -569,30 +622,32 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
       dim3 g(static_cast<unsigned>(N_pad / awq::kQuantRowsPerCta),
              static_cast<unsigned>(K / awq::kGroup), static_cast<unsigned>(na));
       if (bits == 4)
-        awq::search_build_error_kernel<4><<<g, 256, 0, st>>>(w, N, K, N_pad, Sa, Ia, E);
+        awq::search_build_error_kernel<4><<<g, 256, 0, st>>>(w, N, K, N_pad, Sa, Ia, rms, E);
       else
-        awq::search_build_error_kernel<3><<<g, 256, 0, st>>>(w, N, K, N_pad, Sa, Ia, E);
+        awq::search_build_error_kernel<3><<<g, 256, 0, st>>>(w, N, K, N_pad, Sa, Ia, rms, E);
       if ((s = launch_status()) != AWQ_OK) return s;
     }
     {
       awq::TcArgs args{};
-      args.M = M;
+      args.M = lay.gram ? K : M;
       args.N = N;
       args.N_pad = N_pad;
       args.K = K;
       args.row_part = part;
       args.m_tiles = m_tiles;
       args.k_splits = 1;
-      s = launch_tc_bn<ASrc::kSplit16, Epi::kRowSumSq>(X, M, E,
-                                                    na * N_pad, args, st);
+      args.E2 = E;
+      s = lay.gram ? launch_tc<kGramBN, ASrc::kGram, Epi::kGramDot>(G2, K, E, na * N_pad, args, st)
+                   : launch_tc_bn<ASrc::kSplit16, Epi::kRowSumSq>(X, M, E, na * N_pad, args, st);
       if (s != AWQ_OK) return s;
     }
     {
       const int64_t n = static_cast<int64_t>(na) * N;
       awq::search_row_loss_kernel<<<static_cast<unsigned>((n + awq::kReduceThreads - 1) /
                                                           awq::kReduceThreads),
-                                    awq::kReduceThreads, 0, st>>>(part, N, N_pad, na, m_tiles,
-                                                                  rl + static_cast<int64_t>(a0) * N);
+                                    awq::kReduceThreads, 0, st>>>(
+          part, N, N_pad, na, m_tiles, lay.gram ? static_cast<double>(M) : 1.0,
+          rl + static_cast<int64_t>(a0) * N);
       if ((s = launch_status()) != AWQ_OK) return s;
     }
   }
@@ -630,9 +685,9 @@ awq_status awq_silu_mul_gemm(const awq_f16* X, int64_t M, const awq_f16* W_gate,
 // ------------------------------------------------------------------ GEMM
 size_t awq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits) {
   if (M <= 0 || K <= 0 || N <= 0) return 0;
-  // the decode kernels need none; 8 < M <= 16 with an X too large for the streaming kernel
-  // takes the tensor-core path below
-  if (M <= 16 && bits == 4 && (M <= 8 || gemv_stream_fits(M, N, K))) return 0;
+  // the decode kernels need none; a call the streaming kernel cannot take (8 < M <= 16 with
+  // an X too large for it, or 3 bits with N % 16 != 0) takes the tensor-core path below
+  if (M <= 16 && (gemv_stream_fits(M, N, K) || (bits == 4 && M <= 8))) return 0;
   const int splits = splitk_for(M, N, K);
   return splits > 1 ? align256(static_cast<size_t>(splits) * M * N * sizeof(float)) : 0;
 }
@@ -655,12 +710,12 @@ awq_status awq_gemm_w4a16(const awq_f16* X, int64_t M, const uint32_t* qweight,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const __half* sc = reinterpret_cast<const __half*>(scales);
 
-  if (M <= 16 && bits == 4) {
-    awq_status r = launch_gemv_stream(X, M, qweight, sc, zeros, N, K, inv_s, flags, Y, st);
+  if (M <= 16) {
+    awq_status r = launch_gemv_stream(X, M, qweight, sc, zeros, N, K, bits, inv_s, flags, Y, st);
     if (r != AWQ_ERR_UNSUPPORTED) return r;
-    // the streaming kernel cannot hold X (or N % 16 != 0): register streaming for fp16 with
-    // M <= 8, the tensor-core path below otherwise
-    if (M <= 8 && !bf16) {
+    // the streaming kernel cannot hold X (or N % 16 != 0): register streaming for fp16 4-bit
+    // with M <= 8, the tensor-core path below otherwise
+    if (M <= 8 && !bf16 && bits == 4) {
       const unsigned grid = static_cast<unsigned>((N + awq::kGemvRows - 1) / awq::kGemvRows);
       awq::gemv_w4a16_kernel<1><<<grid, awq::kGemvWarps * 32, 0, st>>>(
           reinterpret_cast<const __half*>(X), static_cast<int>(M), qweight, sc, zeros, N, K,

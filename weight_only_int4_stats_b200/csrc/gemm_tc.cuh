@@ -58,18 +58,32 @@ constexpr int kTcSmemMax = 232448;  // dynamic shared memory per CTA on sm_100
 // and the epilogue combines them in fp32.
 // kPair16: two fp16 weights of the same shape (a gated MLP's gate_proj and up_proj); the
 // same rows of both are the two A parts, each with its own accumulator.
-enum class ASrc : int { kPacked4 = 0, kPacked3 = 1, kSplit16 = 2, kPair16 = 3 };
+// kFp16x1: one plain fp16 matrix (the Gram matrix X^T X of the calibration tokens).
+// kGram: the search's error operand (two parts, as kSplit16) against the normalised Gram
+// matrix, itself in two fp16 parts [hi | lo] as the B operand: per 16-k step the MMAs
+// A_hi B_hi -> accumulator 0 and A_hi B_lo, A_lo B_hi -> accumulator 1, recombined as
+// D = D_0 + 2^-12 D_1 (the lo x lo product, 2^-24 relative, is left out).
+enum class ASrc : int { kPacked4 = 0, kPacked3 = 1, kSplit16 = 2, kPair16 = 3, kFp16x1 = 4,
+                        kGram = 5 };
 // kStoreY: fp16 Y (or fp32 split-K partials); kRowSumSq: per-row sums of squares of the
-// recombined two-part product; kSiluMul: fp16 H = silu(D_0) * D_1 of the two accumulators.
-enum class Epi : int { kStoreY = 0, kRowSumSq = 1, kSiluMul = 2 };
+// recombined two-part product; kSiluMul: fp16 H = silu(D_0) * D_1 of the two accumulators;
+// kStoreF32: the fp32 product itself (the Gram matrix); kGramDot: per-row sums of
+// D[n][j] * e'[n][j], the recombined product times the row's own error operand.
+enum class Epi : int { kStoreY = 0, kRowSumSq = 1, kSiluMul = 2, kStoreF32 = 3, kGramDot = 4 };
 
 template <int BN, ASrc kA>
 struct TcLayout {
   static constexpr bool kPk = kA == ASrc::kPacked4 || kA == ASrc::kPacked3;
+  static constexpr int kXParts = kA == ASrc::kGram ? 2 : 1;   // B tiles per stage
+  static constexpr int kAParts = (kPk || kA == ASrc::kFp16x1) ? 1 : 2;   // A tiles (and
+                                                                       // accumulators) per stage
+  static constexpr int kXPartBytes = BN * kTcBK * 2;
+  static constexpr int kXBytes = kXParts * kXPartBytes;
   static constexpr int kStages =
-      !kPk ? (BN >= 256 ? 3 : BN >= 128 ? 4 : BN >= 64 ? 5 : 6) : (BN >= 256 ? 4 : BN >= 64 ? 5 : 6);
-  static constexpr int kXBytes = BN * kTcBK * 2;
-  static constexpr int kAParts = kPk ? 1 : 2;            // A tiles (and accumulators) per stage
+      kA == ASrc::kGram ? (BN >= 256 ? 2 : BN >= 128 ? 3 : 4)
+      : kA == ASrc::kFp16x1 ? (BN >= 256 ? 4 : 6)
+      : !kPk ? (BN >= 256 ? 3 : BN >= 128 ? 4 : BN >= 64 ? 5 : 6)
+             : (BN >= 256 ? 4 : BN >= 64 ? 5 : 6);
   static constexpr int kAPartBytes = kTcBM * kTcBK * 2;
   static constexpr int kABytes = kAParts * kAPartBytes;
   // packed source: kPG groups (2 kPG stages) per ring slot
@@ -118,6 +132,8 @@ struct TcArgs {
   int sz_tma;           // packed source: scales and zeros arrive by TMA with the packed group
                         // (needs N % 16 == 0); else the builders load them from global memory
   const float* inv_s;   // packed source: NULL, or [K] factors folded into the weights
+  float* G;             // kStoreF32: [rows_total, M] fp32 output (the Gram matrix)
+  const __half* E2;     // kGramDot: the error operand [rows_total, 2K] the epilogue reads
 };
 
 // Grouped tile order: consecutive work units sweep the token tiles of a group of
@@ -250,6 +266,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   static_assert(!kPacked || L::kPSlots >= 2, "packed ring needs two slots");
   static_assert(kEpi != Epi::kRowSumSq || kA == ASrc::kSplit16,
                 "the sum-of-squares epilogue recombines the two-part error operand");
+  static_assert(kEpi != Epi::kStoreF32 || kA == ASrc::kFp16x1, "the Gram product");
+  static_assert(kEpi != Epi::kGramDot || kA == ASrc::kGram, "the Gram-form loss");
   static_assert(kEpi != Epi::kSiluMul || kA == ASrc::kPair16,
                 "the SiLU epilogue combines the gate and up accumulators");
   static_assert(kEpi != Epi::kStoreY || kPacked, "fp16 Y comes from the packed sources");
@@ -321,7 +339,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           mbar_arrive_expect_tx(&full[s], L::kTxBytes);
           tma_load_2d(smem + L::kXOff + s * L::kXBytes, &tmap_x, &full[s], kb * kTcBK,
                       static_cast<int32_t>(m0));
-          if (kA == ASrc::kSplit16) {
+          if (kA == ASrc::kGram)   // the lo part of the normalised Gram matrix
+            tma_load_2d(smem + L::kXOff + s * L::kXBytes + L::kXPartBytes, &tmap_x, &full[s],
+                        static_cast<int32_t>(args.K) + kb * kTcBK, static_cast<int32_t>(m0));
+          if (kA == ASrc::kFp16x1) {
+            tma_load_2d(smem + L::kAOff + s * L::kABytes, &tmap_a, &full[s], kb * kTcBK,
+                        static_cast<int32_t>(row0));
+          } else if (kA == ASrc::kSplit16 || kA == ASrc::kGram) {
             uint8_t* a = smem + L::kAOff + s * L::kABytes;
             tma_load_2d(a, &tmap_a, &full[s], kb * kTcBK, static_cast<int32_t>(row0));
             tma_load_2d(a + L::kAPartBytes, &tmap_a, &full[s],
@@ -360,11 +384,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t x_base = smem_u32(smem + L::kXOff + s * L::kXBytes);
 #pragma unroll
           for (int kk = 0; kk < kTcBK / 16; ++kk) {
+            const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
+            if (kA == ASrc::kGram) {
+              // A_hi B_hi -> D_0; A_hi B_lo + A_lo B_hi -> D_1
+              const uint64_t ah = sw128_kmajor_desc(a_base + kk * 32);
+              const uint64_t al = sw128_kmajor_desc(a_base + L::kAPartBytes + kk * 32);
+              const uint64_t bh = sw128_kmajor_desc(x_base + kk * 32);
+              const uint64_t bl = sw128_kmajor_desc(x_base + L::kXPartBytes + kk * 32);
+              tc_mma_f16(d_tmem, ah, bh, idesc, acc);
+              tc_mma_f16(d_tmem + static_cast<uint32_t>(BN), ah, bl, idesc, acc);
+              tc_mma_f16(d_tmem + static_cast<uint32_t>(BN), al, bh, idesc, 1u);
+            } else {
 #pragma unroll
-            for (int part = 0; part < L::kAParts; ++part)   // part p: A tile p -> accumulator p
-              tc_mma_f16(d_tmem + static_cast<uint32_t>(part * BN),
-                         sw128_kmajor_desc(a_base + part * L::kAPartBytes + kk * 32),
-                         sw128_kmajor_desc(x_base + kk * 32), idesc, (i | kk) != 0 ? 1u : 0u);
+              for (int part = 0; part < L::kAParts; ++part)   // part p: A tile p -> accumulator p
+                tc_mma_f16(d_tmem + static_cast<uint32_t>(part * BN),
+                           sw128_kmajor_desc(a_base + part * L::kAPartBytes + kk * 32),
+                           sw128_kmajor_desc(x_base + kk * 32), idesc, acc);
+            }
           }
           tc_commit(&empty[s]);
           if (++s == S) { s = 0; ph ^= 1; }
@@ -518,6 +554,45 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               }
             }
           }
+        } else if (kEpi == Epi::kStoreF32) {
+          // Slices of the contraction (k_splits) of one output tile are the consecutive units of
+          // one CTA (the grid is one CTA per tile), so slice s > 0 adds itself to the sum of
+          // slices 0..s-1 with one rounded fp32 add, in order: short accumulation chains in
+          // TMEM, a fixed summation order, no race.
+          if (arow < args.rows_total && unit_ok) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int64_t m = m0 + col + j;
+              if (m < args.M) {
+                float* gp = args.G + arow * args.M + m;
+                *gp = t.ksplit == 0 ? __uint_as_float(v[j]) : __fadd_rn(*gp, __uint_as_float(v[j]));
+              }
+            }
+          }
+        } else if (kEpi == Epi::kGramDot) {
+          // sum_j (D_0 + 2^-12 D_1)[n][j] * (hi + 2^-12 lo)[n][j] over the tile's 16 columns
+          uint32_t vl[16];
+          tmem_ld_32x32b_x16(taddr + BN + col, vl);
+          tmem_ld_wait();
+          if (arow < args.rows_total && unit_ok) {
+            const __half* er = args.E2 + arow * 2 * args.K + m0 + col;
+            const uint4* eh = reinterpret_cast<const uint4*>(er);
+            const uint4* el = reinterpret_cast<const uint4*>(er + args.K);
+            const uint4 h4[2] = {eh[0], eh[1]}, l4[2] = {el[0], el[1]};
+            const uint32_t hw[8] = {h4[0].x, h4[0].y, h4[0].z, h4[0].w, h4[1].x, h4[1].y, h4[1].z, h4[1].w};
+            const uint32_t lw[8] = {l4[0].x, l4[0].y, l4[0].z, l4[0].w, l4[1].x, l4[1].y, l4[1].z, l4[1].w};
+            float part = 0.0f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float2 hf = __half22float2(u32_as_h2(hw[q])), lf = __half22float2(u32_as_h2(lw[q]));
+              const float e0 = fmaf(lf.x, 0x1p-12f, hf.x), e1 = fmaf(lf.y, 0x1p-12f, hf.y);
+              const float d0 = fmaf(__uint_as_float(vl[2 * q]), 0x1p-12f, __uint_as_float(v[2 * q]));
+              const float d1 = fmaf(__uint_as_float(vl[2 * q + 1]), 0x1p-12f, __uint_as_float(v[2 * q + 1]));
+              part = fmaf(d0, e0, part);
+              part = fmaf(d1, e1, part);
+            }
+            sumsq += static_cast<double>(part);
+          }
         } else if (kEpi == Epi::kSiluMul) {
           // h = silu(g) * u = g * u / (1 + exp(-g)), g and u the gate and up accumulators
           uint32_t vu[16];
@@ -546,7 +621,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           sumsq += static_cast<double>(part);
         }
       }
-      if (kEpi == Epi::kRowSumSq && unit_ok && AWQ_IN_BOUNDS(arow < args.rows_total))
+      if ((kEpi == Epi::kRowSumSq || kEpi == Epi::kGramDot) && unit_ok &&
+          AWQ_IN_BOUNDS(arow < args.rows_total))
         args.row_part[static_cast<int64_t>(t.m_tile) * args.rows_total + arow] = sumsq;
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);            // the MMA may overwrite this accumulator

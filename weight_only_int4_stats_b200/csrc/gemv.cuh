@@ -204,74 +204,95 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_w4a16_kernel(
 namespace awq {
 
 // ---------------------------------------------------------------------------------------
-// Streaming decode GEMM (the decode path for M <= 16 when X fits in shared memory; an
-// 8 < M <= 16 call whose X does not fit takes the tensor-core GEMM instead).
+// Streaming decode GEMM (the decode path for M <= 16; N in whole 16-row tiles and X within
+// one CTA's shared memory).
 //
 // Persistent: the grid is one CTA per SM (as many as there are 16-row tiles, at most) and
 // CTA b owns the contiguous range of whole 16-row tiles [b*T/P, (b+1)*T/P), so no output is
 // split across CTAs and the result does not depend on the grid. One producer thread walks
-// the CTA's (tile, 2048-k chunk) units and streams each unit's packed weights
-// ([16 rows, 256 words] = 16 KB), fp16 scales and uint8 zeros ([16 groups, 16 rows]) with
-// TMA into a shared-memory ring of up to kGSMaxSlots slots.
+// the CTA's (tile, 2048-k chunk) units and streams each unit's packed weights (16 rows x
+// 1 KB at 4 bits, 768 B at 3 bits), fp16 scales and uint8 zeros ([16 groups, 16 rows]) with
+// TMA into a shared-memory ring. The packed weights arrive as 128-byte-wide boxes with the
+// 128-byte swizzle (16-byte chunk c of row r of a box at chunk c ^ (r % 8)), so the consumers'
+// 16-byte reads of eight rows at once hit eight different bank groups: without it the rows,
+// 1 KB apart, all map to the same banks. A quarter-warp's eight 16-byte reads come from two
+// rows and four chunks; lane row r reads weight row rho(r) = r/2 + 4(r%2) of the box (and
+// rho(r) + 8), so the two rows of a quarter-warp differ in the swizzle's bit 2 and their
+// chunks land in opposite halves of the 128-byte line: eight reads, eight bank groups, one
+// wavefront. The MMA's row r is then weight row rho(r) of the tile.
 //
 // Back-to-back launches overlap (programmatic dependent launch). A CTA needs at most half of
 // an SM's shared memory, so the next GEMM's CTAs become resident beside this one's as soon as
-// every CTA of this grid has passed griddepcontrol.wait (the point where the launch of the
-// next grid is allowed). Before its own griddepcontrol.wait, a CTA touches no output and no
-// activation: it issues L2 prefetches of its weight rows (coherent with writes of the
-// preceding kernel, so always safe) and, when the caller states that the weights are not
-// written by the kernel launched just before (kGemvWeightsReady), TMA-loads the first ring
-// slots so that this GEMM's weights stream while the preceding kernel still runs. X
-// ([M, K], small at decode) is bulk-copied into shared memory after the wait.
+// every CTA of this grid has passed griddepcontrol.wait (where the next launch is allowed).
+// Before the wait a CTA touches no output and no activation: it issues L2 prefetches of its
+// weight rows (coherent with writes of the preceding kernel, so always safe) and, when the
+// caller states that the weights are not written by the kernel launched just before
+// (kGemvWeightsReady), TMA-loads the first ring slots.
 //
-// kCW consumer warps each take 16 / kCW of the unit's sixteen 128-wide groups, with
-// register-only dequantization feeding mma.sync m16n8k16 (weights as the 16-row A operand,
-// activations as the 8-column B operand). A warp copies its packed words, scales and zero
-// points of the unit to registers and releases the ring slot before the arithmetic, so the
-// producer can refill it at once. Two dequantization forms:
+// After the wait the consumer warps stage X ([M, K], small at decode) from global memory into
+// shared memory in the order the MMA's B fragments read it -- [group][8-k chunk j][token][32-k
+// quarter c] of 16 bytes -- so one fragment read is 64 contiguous bytes at M = 1. Eight
+// consumer warps each take two of a unit's sixteen 128-wide groups, with register-only
+// dequantization feeding mma.sync m16n8k16 (weights as the 16-row A operand, activations as
+// the 8-column B operand). A warp copies its packed words, scales and zero points of the unit
+// to registers and releases the ring slot before the arithmetic. Two dequantization forms:
 //  * M = 1 (kOffset): a mask-and-or with 0x6400 turns the nibble pair (k0, k1) of a word
 //    into the exact fp16 values (1024 + q0, 1024 + q1) and the pair (k2, k3), stored 4 bits
 //    higher, into (1024 + 16 q2, 1024 + 16 q3) (the same after a shift by 8 for k4..k7);
 //    these go to the MMA unchanged against X staged with columns k%8 in {2,3,6,7} divided by
 //    16 (exact in fp16), so per group the MMA returns sum_k x_k q_k + C1 with
 //    C1 = 1024 * sum_k xs_k; with C2 = sum_k x_k the group adds s * (mma - C1 - z C2).
-//    The staging and C1, C2 are one pass over X per CTA. Five integer operations per
-//    packed word; the fp32 cancellation of the 1024 offset keeps about 13 significant bits
-//    of each group sum.
+//    Five integer operations per packed word; the fp32 cancellation of the 1024 offset keeps
+//    about 13 significant bits of each group sum. (3-bit codes and bf16 have one raw pair
+//    form, base 1024 or 128, so X is staged undivided and C1 = base * C2.)
 //  * M > 1: one fp16 subtract (or multiply-add) per pair leaves the exact q - z first.
 // Each group's eight MMAs run as four independent accumulator chains. At the end of a tile
-// the consumer warps' partial sums are added in a fixed warp order and stored as fp16.
+// the consumer warps' partial sums are added in a fixed warp order and stored.
 // ---------------------------------------------------------------------------------------
 constexpr int kG4Groups = 16;                      // groups per unit
 constexpr int kG4KC = kG4Groups * kGroup;          // k per unit (2048)
-constexpr int kG4WBytes = kGemvRows * (kG4KC / 2);             // 16384
+constexpr int kG4Warps = 8;                        // consumer warps (two groups each per unit)
+constexpr int kG4Threads = (kG4Warps + 1) * 32;    // + one producer warp
+constexpr int kG4WSlot = kGemvRows * kG4KC / 2;    // ring slot stride of the packed codes (16 KB)
 constexpr int kG4SBytes = kG4Groups * kGemvRows * 2;           // 512
 constexpr int kG4ZBytes = kG4Groups * kGemvRows;               // 256
-constexpr int kG4SlotBytes = kG4WBytes + kG4SBytes + kG4ZBytes; // 17152 (multiple of 128)
+constexpr int kG4Box = kGemvRows * 128;                        // one swizzled box: 16 rows x 128 B
 constexpr int kGSMaxSlots = 6;
 
 // Flag bits of the decode launch (awq_gemm_w4a16's flags).
 constexpr unsigned kGemvWeightsReady = 1u;
 
+// Shared memory, from a 1024-byte aligned base (the swizzle's period): the packed-code slots,
+// then per slot its scales and zero points, the staged X, the per-(group, token) sums, the
+// barriers and the tile-end reduction buffer.
 struct G4Smem {
+  int slots;     // ring depth
   int x_bytes;   // M * K * 2, rounded up to 128
   int c_bytes;   // C1/C2 per (group, token)
-  int slots;     // ring depth
-  int cw;        // consumer warps
-  __host__ __device__ int c_off() const { return x_bytes; }
-  __host__ __device__ int slot_off() const { return x_bytes + c_bytes; }
-  __host__ __device__ int bar_off() const { return slot_off() + slots * kG4SlotBytes; }
+  __host__ __device__ int sz_off() const { return slots * kG4WSlot; }
+  __host__ __device__ int x_off() const { return sz_off() + slots * (kG4SBytes + kG4ZBytes); }
+  __host__ __device__ int c_off() const { return x_off() + x_bytes; }
+  __host__ __device__ int bar_off() const { return c_off() + c_bytes; }
   __host__ __device__ int red_off() const { return bar_off() + (2 * kGSMaxSlots + 2) * 8; }
-  __host__ __device__ int total(int n_tiles) const { return red_off() + cw * n_tiles * 4 * 32 * 4; }
-  __host__ __device__ static G4Smem make(int M, int64_t K, int n_tiles, int slots, int cw) {
+  // + 1024 bytes of slack for aligning the base
+  __host__ __device__ int total(int n_tiles) const {
+    return red_off() + kG4Warps * n_tiles * 4 * 32 * 4 + 1024;
+  }
+  __host__ __device__ static G4Smem make(int M, int64_t K, int n_tiles, int slots) {
     G4Smem l;
+    l.slots = slots;
     l.x_bytes = static_cast<int>((static_cast<int64_t>(M) * K * 2 + 127) / 128 * 128);
     l.c_bytes = static_cast<int>(((K / kGroup) * 8 * n_tiles * 2 * 4 + 127) / 128 * 128);
-    l.slots = slots;
-    l.cw = cw;
     return l;
   }
 };
+
+// Byte offset of packed word w (0..kG4KC*bits/32 - 1 of a unit's row) of row r in a slot of
+// swizzled 128-byte boxes.
+__device__ __forceinline__ uint32_t g4_word_offset(int r, int w) {
+  return static_cast<uint32_t>((w >> 5) * kG4Box + r * 128 + ((((w >> 2) & 7) ^ (r & 7)) << 4) +
+                               (w & 3) * 4);
+}
 
 // One packed word -> the raw fp16 pairs (1024+q0,1024+q1), (1024+16q2,1024+16q3),
 // (1024+q4,1024+q5), (1024+16q6,1024+16q7); with bf16 activations the raw bf16 pairs
@@ -293,6 +314,23 @@ __device__ __forceinline__ void raw_word(uint32_t w, uint32_t (&v)[4]) {
   }
 }
 
+// 3-bit: the raw pairs (base + q) of chunk i (k = 8i..8i+7) of a 32-k block whose low-bit words
+// are w0 (offsets 0..15) / w1 (16..31) and whose bit-2 word is w2 (layout of the 3-bit packing:
+// the pair's two crumbs at 2-bit field 4(i%2) + e of its low word, its two high bits at bits
+// 4i + e and 4i + e + 16 of w2); base 1024 (fp16, 0x6400) or 128 (bf16, 0x4300).
+template <bool kBf16>
+__device__ __forceinline__ void raw3_chunk(uint32_t w0, uint32_t w1, uint32_t w2, int i,
+                                           uint32_t (&v)[4]) {
+  const uint32_t wlo = i < 2 ? w0 : w1;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int pp = 4 * (i & 1) + e, hb = 4 * i + e;
+    const uint32_t lo = lop3_and_or(wlo >> (2 * pp), 0x00030003u, kBf16 ? 0x43004300u : 0x64006400u);
+    const uint32_t hs = hb >= 2 ? (w2 >> (hb - 2)) : (w2 << (2 - hb));
+    v[e] = lop3_and_or(hs, 0x00040004u, lo);
+  }
+}
+
 // The exact pairs (q - z) in bf16: the raw pairs minus (128 + z).
 __device__ __forceinline__ void dequant_word_qz_bf16(uint32_t w, uint32_t bias, uint32_t (&out)[4]) {
   raw_word<true>(w, out);
@@ -300,22 +338,29 @@ __device__ __forceinline__ void dequant_word_qz_bf16(uint32_t w, uint32_t bias, 
   for (int i = 0; i < 4; ++i) out[i] = b2_as_u32(__hsub2(u32_as_b2(out[i]), u32_as_b2(bias)));
 }
 
-template <int kNTiles, bool kOffset, int kCW, bool kBf16 = false>
-__global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
+template <int kNTiles, bool kOffset, bool kBf16 = false, int kBits = 4>
+__global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
     const __grid_constant__ CUtensorMap tmap_z, const uint32_t* __restrict__ qweight,
     const act_t<kBf16>* __restrict__ X, int M, int64_t N, int64_t K,
     const float* __restrict__ inv_s, act_t<kBf16>* __restrict__ Y, G4Smem lay, unsigned flags) {
-  static_assert(kG4Groups % kCW == 0, "consumer warps must divide the unit's groups");
-  constexpr int kGPW = kG4Groups / kCW;   // groups per consumer warp and unit
+  static_assert(kBits == 4 || kBits == 3, "4- or 3-bit codes");
   constexpr int kTok = 8 * kNTiles;
-  extern __shared__ __align__(128) uint8_t smem[];
-  act_t<kBf16>* xs = reinterpret_cast<act_t<kBf16>*>(smem);
+  constexpr int kRowW = kG4KC * kBits / 32;            // packed words of one row in a unit
+  constexpr int kBoxes = kRowW / 32;                   // 128-byte boxes per unit (8 or 6)
+  constexpr uint32_t kTx = kGemvRows * kRowW * 4 + kG4SBytes + kG4ZBytes;
+  // M = 1 with fp16 and 4 bits stages columns k%8 in {2,3,6,7} divided by 16 (the nibbles
+  // stored 4 bits higher come out as 1024 + 16q); every other form has one raw pair form
+  constexpr bool kDiv16 = !kBf16 && kBits == 4;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* wslots = smem;
+  uint8_t* szslots = smem + lay.sz_off();
+  act_t<kBf16>* xs = reinterpret_cast<act_t<kBf16>*>(smem + lay.x_off());   // [G][4][M][4] x 8
   float* cc = reinterpret_cast<float*>(smem + lay.c_off());
-  uint8_t* slots = smem + lay.slot_off();
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bar_off());
   uint64_t* empty = full + kGSMaxSlots;
-  uint64_t* xfull = empty + kGSMaxSlots;
   float* red = reinterpret_cast<float*>(smem + lay.red_off());
   const int S = lay.slots;
 
@@ -332,14 +377,13 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kCW * 32);
+      mbar_init(&empty[i], kG4Warps * 32);
     }
-    mbar_init(xfull, 1);
     fence_barrier_init();
   }
   __syncthreads();
 
-  if (warp == kCW) {
+  if (warp == kG4Warps) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       tma_prefetch_desc(&tmap_w);
@@ -350,12 +394,15 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
       int64_t tile = t0;
       auto issue = [&]() {
         if (!AWQ_IN_BOUNDS(slot < S && tile < t1 && chunk < C)) return;
-        uint8_t* sb = slots + slot * kG4SlotBytes;
-        mbar_arrive_expect_tx(&full[slot], kG4SlotBytes);
+        uint8_t* wb = wslots + slot * kG4WSlot;
+        uint8_t* sz = szslots + slot * (kG4SBytes + kG4ZBytes);
+        mbar_arrive_expect_tx(&full[slot], kTx);
         const int32_t row = static_cast<int32_t>(tile * kGemvRows);
-        tma_load_2d(sb, &tmap_w, &full[slot], chunk * (kG4KC / 8), row);
-        tma_load_2d(sb + kG4WBytes, &tmap_s, &full[slot], row, chunk * kG4Groups);
-        tma_load_2d(sb + kG4WBytes + kG4SBytes, &tmap_z, &full[slot], row, chunk * kG4Groups);
+#pragma unroll
+        for (int b = 0; b < kBoxes; ++b)
+          tma_load_2d(wb + b * kG4Box, &tmap_w, &full[slot], chunk * kRowW + b * 32, row);
+        tma_load_2d(sz, &tmap_s, &full[slot], row, chunk * kG4Groups);
+        tma_load_2d(sz + kG4SBytes, &tmap_z, &full[slot], row, chunk * kG4Groups);
         if (++slot == S) { slot = 0; ph ^= 1; }
         if (++chunk == C) { chunk = 0; ++tile; }
       };
@@ -366,7 +413,7 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
         for (; u < n_early; ++u) issue();
       }
       {   // HBM -> L2 for this CTA's weight rows (one contiguous range)
-        const int64_t row_bytes = K / 2;
+        const int64_t row_bytes = K * kBits / 8;
         const int64_t r0 = t0 * kGemvRows, r1 = t1 * kGemvRows < N ? t1 * kGemvRows : N;
         const uint8_t* wrow = reinterpret_cast<const uint8_t*>(qweight) + r0 * row_bytes;
         const int64_t bytes = (r1 - r0) * row_bytes;
@@ -376,8 +423,6 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
       pdl_wait();
       // every kernel before this one has completed: the next grid may now be scheduled
       pdl_launch_dependents();
-      mbar_arrive_expect_tx(xfull, static_cast<uint32_t>(M * K * 2));
-      bulk_load_1d(xs, X, static_cast<uint32_t>(M * K * 2), xfull);
       for (; u < units; ++u) {
         if (!mbar_wait(&empty[slot], ph ^ 1)) break;
         issue();
@@ -387,69 +432,67 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
   }
 
   // ------------------------------------------------------------------ consumers
-  // A timed-out wait clears `ok`; the warp then skips further waits and arithmetic but still
-  // runs every named barrier, so the consumer warps cannot deadlock one another.
   const int r = lane >> 2, c = lane & 3;
-  bool ok = __all_sync(0xffffffffu, mbar_wait(xfull, 0));
-  if (kOffset) {
-    // One pass over X: x <- fp16(x * inv_s), columns k%8 in {2,3,6,7} divided by 16 (exact
-    // in fp16), and per (group, token < M) C1 = 1024 * sum(xs) and C2 = sum(x) from the staged
-    // values; tokens >= M get zeros. (bf16: x <- bf16(x * inv_s), no division, C2 = sum(x)
-    // and C1 = 128 * C2.) 8 threads per (group, token) pair, 2 chunks of 8 each, 4 pairs per
-    // warp and pass, three xor-shuffles.
+  const int rw = (r >> 1) + 4 * (r & 1);   // weight row (of the tile) of the MMA's row r
+  pdl_wait();   // X may be the preceding kernel's output
+  // Stage X: x <- x * inv_s (kDiv16: columns k%8 in {2,3,6,7} / 16), in B-fragment order, and
+  // for M = 1 per-(group, token) C1 / C2. 8 threads per (group, token) pair, each 16
+  // consecutive values (two 8-value chunks), three xor-shuffles.
+  {
     const int sub = lane & 7;
     const int npairs = G * M;
     const __half2 sixteenth = __float2half2_rn(0.0625f);
-    for (int base = warp * 4; base < npairs; base += kCW * 4) {
+    for (int base = warp * 4; base < npairs; base += kG4Warps * 4) {
       const int pr = base + (lane >> 3);
-      const bool live = ok && pr < npairs;
+      const bool live = pr < npairs;
       const int g = live ? pr / M : 0, m = live ? pr % M : 0;
-      uint4* src = reinterpret_cast<uint4*>(xs + m * Ki + g * kGroup + 16 * sub);
       float c1 = 0.0f, c2 = 0.0f;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        uint4 v = live ? src[h] : make_uint4(0u, 0u, 0u, 0u);
-        if (inv_s != nullptr && live) {
-          const int k = g * kGroup + 16 * sub + 8 * h;
+        const int koff = 16 * sub + 8 * h;              // offset inside the group
+        const int k = g * kGroup + koff;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (live) v = *reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * Ki + k);
+        if (inv_s != nullptr && live)
           v = scale8<kBf16>(v, *reinterpret_cast<const float4*>(inv_s + k),
                             *reinterpret_cast<const float4*>(inv_s + k + 4));
-        }
-        if constexpr (!kBf16) {
+        if (kOffset && kDiv16) {
           v.y = h2_as_u32(__hmul2(u32_as_h2(v.y), sixteenth));
           v.w = h2_as_u32(__hmul2(u32_as_h2(v.w), sixteenth));
         }
-        if (live) src[h] = v;
-        const float2 lx = act2_to_float2<kBf16>(v.x), hy = act2_to_float2<kBf16>(v.y);
-        const float2 lz = act2_to_float2<kBf16>(v.z), hw = act2_to_float2<kBf16>(v.w);
-        const float lo = (lx.x + lx.y) + (lz.x + lz.y), hi = (hy.x + hy.y) + (hw.x + hw.y);
-        c1 += lo + hi;
-        c2 += kBf16 ? lo + hi : lo + 16.0f * hi;
+        const int cq = koff >> 5, jq = (koff >> 3) & 3;   // 32-k quarter, 8-k chunk
+        if (live && AWQ_IN_BOUNDS(((g * 4 + jq) * M + m) * 4 + cq < G * 4 * M * 4))
+          reinterpret_cast<uint4*>(xs)[((g * 4 + jq) * M + m) * 4 + cq] = v;
+        if (kOffset) {
+          const float2 lx = act2_to_float2<kBf16>(v.x), hy = act2_to_float2<kBf16>(v.y);
+          const float2 lz = act2_to_float2<kBf16>(v.z), hw = act2_to_float2<kBf16>(v.w);
+          const float lo = (lx.x + lx.y) + (lz.x + lz.y), hi = (hy.x + hy.y) + (hw.x + hw.y);
+          c1 += lo + hi;
+          c2 += kDiv16 ? lo + 16.0f * hi : lo + hi;
+        }
       }
+      if (kOffset) {
 #pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
-        c1 += __shfl_xor_sync(0xffffffffu, c1, o);
-        c2 += __shfl_xor_sync(0xffffffffu, c2, o);
-      }
-      if (sub == 0 && live) {
-        cc[(g * kTok + m) * 2] = kBf16 ? 128.0f * c2 : 1024.0f * c1;
-        cc[(g * kTok + m) * 2 + 1] = c2;
+        for (int o = 1; o < 8; o <<= 1) {
+          c1 += __shfl_xor_sync(0xffffffffu, c1, o);
+          c2 += __shfl_xor_sync(0xffffffffu, c2, o);
+        }
+        if (sub == 0 && live) {
+          // C1 = base * sum of the staged values (c1 == c2 unless kDiv16)
+          cc[(g * kTok + m) * 2] = kBf16 ? 128.0f * c2 : 1024.0f * c1;
+          cc[(g * kTok + m) * 2 + 1] = c2;
+        }
       }
     }
-    for (int i = threadIdx.x; i < G * kTok; i += kCW * 32)
-      if (i % kTok >= M) { cc[2 * i] = 0.0f; cc[2 * i + 1] = 0.0f; }
-    named_bar_sync(1, kCW * 32);
-  } else if (inv_s != nullptr) {
-    // x <- fp16(x * inv_s) (bf16 for bf16 activations)
-    const int n8 = M * Ki / 8;
-    for (int i = threadIdx.x; ok && i < n8; i += kCW * 32) {
-      const int k = (i * 8) % Ki;
-      reinterpret_cast<uint4*>(xs)[i] =
-          scale8<kBf16>(reinterpret_cast<uint4*>(xs)[i], *reinterpret_cast<const float4*>(inv_s + k),
-                        *reinterpret_cast<const float4*>(inv_s + k + 4));
-    }
-    named_bar_sync(1, kCW * 32);
+    if (kOffset)
+      for (int i = threadIdx.x; i < G * kTok; i += kG4Warps * 32)
+        if (i % kTok >= M) { cc[2 * i] = 0.0f; cc[2 * i + 1] = 0.0f; }
+    named_bar_sync(1, kG4Warps * 32);
   }
 
+  // A timed-out wait clears `ok`; the warp then skips further waits and arithmetic but still
+  // runs every named barrier, so the consumer warps cannot deadlock one another.
+  bool ok = true;
   float total[kNTiles][4];
 #pragma unroll
   for (int t = 0; t < kNTiles; ++t)
@@ -461,32 +504,45 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
   int64_t tile = t0;
   for (int64_t u = 0; u < units; ++u) {
     ok = __all_sync(0xffffffffu, ok && mbar_wait(&full[slot], ph));
-    // Copy this warp's operands of the unit (its groups: packed words of rows r and r + 8,
+    // Copy this warp's operands of the unit (its two groups: packed codes of rows r and r + 8,
     // their scales and zero points) to registers and release the slot at once, so the
     // producer refills it while this unit is computed. Every lane arrives (release
     // semantics), which orders its own shared-memory reads first.
-    const uint8_t* sb = slots + slot * kG4SlotBytes;
-    uint4 wA[kGPW], wB[kGPW];
-    uint32_t zAi[kGPW], zBi[kGPW];
-    float scA[kGPW], scB[kGPW];
+    const uint8_t* wb = wslots + slot * kG4WSlot;
+    const uint8_t* sz = szslots + slot * (kG4SBytes + kG4ZBytes);
+    uint4 wA[2], wB[2];   // 4-bit: words 4c..4c+3 of the group; 3-bit: .x .y .z = the lane's
+                          // 32-k block (low words, bit-2 word)
+    uint32_t zAi[2], zBi[2];
+    float scA[2], scB[2];
 #pragma unroll
-    for (int q = 0; q < kGPW; ++q) {
-      const int gl = kGPW * warp + q;               // group inside the unit
-      const uint8_t* wrow = sb + (gl * 16 + 4 * c) * 4;
-      wA[q] = *reinterpret_cast<const uint4*>(wrow + r * (kG4KC / 2));
-      wB[q] = *reinterpret_cast<const uint4*>(wrow + (r + 8) * (kG4KC / 2));
-      const __half* ss = reinterpret_cast<const __half*>(sb + kG4WBytes) + gl * kGemvRows;
-      const uint8_t* zz = sb + kG4WBytes + kG4SBytes + gl * kGemvRows;
-      zAi[q] = zz[r];
-      zBi[q] = zz[r + 8];
-      scA[q] = __half2float(ss[r]);
-      scB[q] = __half2float(ss[r + 8]);
+    for (int q = 0; q < 2; ++q) {
+      const int gl = 2 * warp + q;               // group inside the unit
+      if constexpr (kBits == 4) {
+        const int w0 = gl * 16 + 4 * c;          // one 16-byte chunk of a swizzled box
+        wA[q] = *reinterpret_cast<const uint4*>(wb + g4_word_offset(rw, w0));
+        wB[q] = *reinterpret_cast<const uint4*>(wb + g4_word_offset(rw + 8, w0));
+      } else {
+        const int w0 = gl * 12 + 3 * c;          // three words, possibly in two chunks
+        wA[q] = make_uint4(*reinterpret_cast<const uint32_t*>(wb + g4_word_offset(rw, w0)),
+                           *reinterpret_cast<const uint32_t*>(wb + g4_word_offset(rw, w0 + 1)),
+                           *reinterpret_cast<const uint32_t*>(wb + g4_word_offset(rw, w0 + 2)), 0u);
+        wB[q] = make_uint4(*reinterpret_cast<const uint32_t*>(wb + g4_word_offset(rw + 8, w0)),
+                           *reinterpret_cast<const uint32_t*>(wb + g4_word_offset(rw + 8, w0 + 1)),
+                           *reinterpret_cast<const uint32_t*>(wb + g4_word_offset(rw + 8, w0 + 2)),
+                           0u);
+      }
+      const __half* ss = reinterpret_cast<const __half*>(sz) + gl * kGemvRows;
+      const uint8_t* zz = sz + kG4SBytes + gl * kGemvRows;
+      zAi[q] = zz[rw];
+      zBi[q] = zz[rw + 8];
+      scA[q] = __half2float(ss[rw]);
+      scB[q] = __half2float(ss[rw + 8]);
     }
     if (ok) mbar_arrive(&empty[slot]);
     if (++slot == S) { slot = 0; ph ^= 1; }
 #pragma unroll
-    for (int q = 0; q < kGPW; ++q) {
-      const int gl = kGPW * warp + q;
+    for (int q = 0; q < 2; ++q) {
+      const int gl = 2 * warp + q;
       const int g = chunk * kG4Groups + gl;
       if (ok && g < G) {
         float acc[kNTiles][4][4];
@@ -498,7 +554,6 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
             for (int i = 0; i < 4; ++i) acc[t][j][i] = 0.0f;
         const uint32_t wordsA[4] = {wA[q].x, wA[q].y, wA[q].z, wA[q].w};
         const uint32_t wordsB[4] = {wB[q].x, wB[q].y, wB[q].z, wB[q].w};
-        const int kx = g * kGroup + 32 * c;
         __half2 loA, hiA, loB, hiB;
         uint32_t bA = 0, bB = 0;   // bf16 bias pairs (128 + z)
         if (!kOffset) {
@@ -515,7 +570,24 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t va[4], vb[4];
-          if (kOffset) {
+          if constexpr (kBits == 3) {
+            raw3_chunk<kBf16>(wA[q].x, wA[q].y, wA[q].z, j, va);
+            raw3_chunk<kBf16>(wB[q].x, wB[q].y, wB[q].z, j, vb);
+            if (!kOffset) {   // minus the bias pair (1024 + z) / (128 + z): the exact q - z
+              const uint32_t ba = ((kBf16 ? 0x4300u : 0x6400u) | zAi[q]) * 0x00010001u;
+              const uint32_t bb = ((kBf16 ? 0x4300u : 0x6400u) | zBi[q]) * 0x00010001u;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                if constexpr (kBf16) {
+                  va[i] = b2_as_u32(__hsub2(u32_as_b2(va[i]), u32_as_b2(ba)));
+                  vb[i] = b2_as_u32(__hsub2(u32_as_b2(vb[i]), u32_as_b2(bb)));
+                } else {
+                  va[i] = h2_as_u32(__hsub2(u32_as_h2(va[i]), u32_as_h2(ba)));
+                  vb[i] = h2_as_u32(__hsub2(u32_as_h2(vb[i]), u32_as_h2(bb)));
+                }
+              }
+            }
+          } else if (kOffset) {
             raw_word<kBf16>(wordsA[j], va);
             raw_word<kBf16>(wordsB[j], vb);
           } else if constexpr (kBf16) {
@@ -529,8 +601,8 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
           for (int t = 0; t < kNTiles; ++t) {
             const int m = r + 8 * t;
             uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-            if (m < M && AWQ_IN_BOUNDS(kx + 8 * j + 8 <= Ki))
-              xv = *reinterpret_cast<const uint4*>(xs + m * Ki + kx + 8 * j);
+            if (m < M && AWQ_IN_BOUNDS(((g * 4 + j) * M + m) * 4 + c < G * 4 * M * 4))
+              xv = reinterpret_cast<const uint4*>(xs)[((g * 4 + j) * M + m) * 4 + c];
             const uint32_t a0[4] = {va[0], vb[0], va[1], vb[1]};
             mma_16816<kBf16>(acc[t][j], a0, xv.x, xv.y);
             const uint32_t a1[4] = {va[2], vb[2], va[3], vb[3]};
@@ -559,7 +631,7 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
     }
 
     if (chunk == C - 1) {
-      // tile complete: fixed-order sum over the consumer warps, fp16 store
+      // tile complete: fixed-order sum over the consumer warps, store
 #pragma unroll
       for (int t = 0; t < kNTiles; ++t)
 #pragma unroll
@@ -567,7 +639,7 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
           red[((warp * kNTiles + t) * 4 + i) * 32 + lane] = total[t][i];
           total[t][i] = 0.0f;
         }
-      named_bar_sync(1, kCW * 32);
+      named_bar_sync(1, kG4Warps * 32);
       if (ok && warp < kNTiles) {
         const int t = warp;
         float v[4];
@@ -575,10 +647,10 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
         for (int i = 0; i < 4; ++i) {
           float sum = 0.0f;
 #pragma unroll
-          for (int w = 0; w < kCW; ++w) sum += red[((w * kNTiles + t) * 4 + i) * 32 + lane];
+          for (int w = 0; w < kG4Warps; ++w) sum += red[((w * kNTiles + t) * 4 + i) * 32 + lane];
           v[i] = sum;
         }
-        const int64_t nA = tile * kGemvRows + r, nB = nA + 8;
+        const int64_t nA = tile * kGemvRows + rw, nB = nA + 8;
         const int m0 = 8 * t + 2 * c, m1 = m0 + 1;
         if (nA < N && AWQ_IN_BOUNDS(tile < t1)) {
           if (m0 < M) Y[static_cast<int64_t>(m0) * N + nA] = float_to_act<kBf16>(v[0]);
@@ -589,7 +661,7 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 2) gemv_stream_kernel(
           if (m1 < M) Y[static_cast<int64_t>(m1) * N + nB] = float_to_act<kBf16>(v[3]);
         }
       }
-      named_bar_sync(1, kCW * 32);
+      named_bar_sync(1, kG4Warps * 32);
     }
     if (++chunk == C) { chunk = 0; ++tile; }
   }

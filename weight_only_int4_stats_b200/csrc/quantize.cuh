@@ -172,12 +172,13 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
 // is exact in fp32, the scaling by a power of 2 too): hi + 2^-12 lo represents e to about 22
 // significant bits instead of fp16's 11. Row n of grid point a is row a * N_pad + n of a
 // [rows, 2K] matrix holding hi in columns 0..K-1 and lo in K..2K-1; rows N..N_pad-1 are
-// written as zeros so that 128-row tiles never straddle two grid points.
+// written as zeros so that 128-row tiles never straddle two grid points. With `rms` (the
+// Gram form of the loss) e is first multiplied by the channel's root mean square rms[k].
 template <int kBits>
 __global__ void __launch_bounds__(256) search_build_error_kernel(
     const __half* __restrict__ W, int64_t N, int64_t K, int64_t N_pad,
     const float* __restrict__ s_table, const float* __restrict__ inv_table,
-    __half* __restrict__ E) {
+    const float* __restrict__ rms, __half* __restrict__ E) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int sub = lane & 7;
@@ -211,6 +212,7 @@ __global__ void __launch_bounds__(256) search_build_error_kernel(
         const float q = code_of<kBits>(w[idx], g);
         const float deq = __fmul_rn(__fsub_rn(q, g.z), g.sc);
         e[u] = __fsub_rn(__fmul_rn(deq, inv[idx]), w_raw[idx]);
+        if (rms != nullptr) e[u] = __fmul_rn(e[u], rms[k0 + idx]);
       }
       const __half2 hi = __floats2half2_rn(e[0], e[1]);
       const float2 hf = __half22float2(hi);
