@@ -232,9 +232,14 @@ awq_status launch_gemv_stream_t(const void* x, int64_t M, const uint32_t* qweigh
                     awq::kG4Groups, awq::kGemvRows, false))
     return AWQ_ERR_CUDA;
   const int64_t tiles = N / awq::kGemvRows;
-  const int64_t sms = num_sms();
+  // Two CTAs per SM (each its own tile range and ring) when both fit, for M <= 8: a CTA's
+  // per-unit chain is latency-bound and a second CTA runs a second chain (measured 21.5
+  // against 23.3 us on the three decode shapes at M = 1). At M <= 16 (two token tiles) one
+  // CTA per SM keeps the ring and X of the larger tiles (two were slower there).
+  const int per_sm = kNTiles == 1 && lay.total(kNTiles) <= kCoResidentSmem ? 2 : 1;
+  const int64_t ctas = static_cast<int64_t>(num_sms()) * per_sm;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(tiles < sms ? tiles : sms));   // one CTA per SM
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles < ctas ? tiles : ctas));
   cfg.blockDim = dim3(awq::kG4Threads);
   cfg.dynamicSmemBytes = static_cast<size_t>(lay.total(kNTiles));
   cfg.stream = st;

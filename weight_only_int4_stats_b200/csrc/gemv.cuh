@@ -229,8 +229,9 @@ namespace awq {
 // caller states that the weights are not written by the kernel launched just before
 // (kGemvWeightsReady), TMA-loads the first ring slots.
 //
-// After the wait the consumer warps stage X ([M, K], small at decode) from global memory into
-// shared memory in the order the MMA's B fragments read it -- [group][8-k chunk j][token][32-k
+// After the wait the consumer warps stage X ([M, K], small at decode; each thread issues all
+// its loads of a round at once) from global memory into shared memory in the order the MMA's
+// B fragments read it -- [group][8-k chunk j][token][32-k
 // quarter c] of 16 bytes -- so one fragment read is 64 contiguous bytes at M = 1. Eight
 // consumer warps each take two of a unit's sixteen 128-wide groups, with register-only
 // dequantization feeding mma.sync m16n8k16 (weights as the 16-row A operand, activations as
@@ -258,6 +259,7 @@ constexpr int kG4SBytes = kG4Groups * kGemvRows * 2;           // 512
 constexpr int kG4ZBytes = kG4Groups * kGemvRows;               // 256
 constexpr int kG4Box = kGemvRows * 128;                        // one swizzled box: 16 rows x 128 B
 constexpr int kGSMaxSlots = 6;
+constexpr int kG4XRound = 4;                       // X chunks per thread per staging round
 
 // Flag bits of the decode launch (awq_gemm_w4a16's flags).
 constexpr unsigned kGemvWeightsReady = 1u;
@@ -436,57 +438,68 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
   const int rw = (r >> 1) + 4 * (r & 1);   // weight row (of the tile) of the MMA's row r
   pdl_wait();   // X may be the preceding kernel's output
   // Stage X: x <- x * inv_s (kDiv16: columns k%8 in {2,3,6,7} / 16), in B-fragment order, and
-  // for M = 1 per-(group, token) C1 / C2. 8 threads per (group, token) pair, each 16
-  // consecutive values (two 8-value chunks), three xor-shuffles.
+  // for M = 1 per-(group, token) C1 / C2. Chunk i (8 values) of X is taken by consumer
+  // thread i % 256 in round i / (256 kG4XRound), every load of a round issued before any is
+  // used; the 16 chunks of one (token, group) are 16 consecutive lanes of one warp (four
+  // xor-shuffles for the sums).
   {
-    const int sub = lane & 7;
-    const int npairs = G * M;
+    const int nch = M * Ki / 8;
+    const int kpr = Ki / 8;   // chunks per token row
+    const int tid = static_cast<int>(threadIdx.x);   // < kG4Warps * 32 (the producer returned)
     const __half2 sixteenth = __float2half2_rn(0.0625f);
-    for (int base = warp * 4; base < npairs; base += kG4Warps * 4) {
-      const int pr = base + (lane >> 3);
-      const bool live = pr < npairs;
-      const int g = live ? pr / M : 0, m = live ? pr % M : 0;
-      float c1 = 0.0f, c2 = 0.0f;
+    for (int base = 0; base < nch; base += kG4Warps * 32 * kG4XRound) {
+      uint4 v[kG4XRound];
+      float4 s0[kG4XRound], s1[kG4XRound];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int koff = 16 * sub + 8 * h;              // offset inside the group
-        const int k = g * kGroup + koff;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (live) v = *reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * Ki + k);
-        if (inv_s != nullptr && live)
-          v = scale8<kBf16>(v, *reinterpret_cast<const float4*>(inv_s + k),
-                            *reinterpret_cast<const float4*>(inv_s + k + 4));
-        if (kOffset && kDiv16) {
-          v.y = h2_as_u32(__hmul2(u32_as_h2(v.y), sixteenth));
-          v.w = h2_as_u32(__hmul2(u32_as_h2(v.w), sixteenth));
-        }
-        const int cq = koff >> 5, jq = (koff >> 3) & 3;   // 32-k quarter, 8-k chunk
-        if (live && AWQ_IN_BOUNDS(((g * 4 + jq) * M + m) * 4 + cq < G * 4 * M * 4))
-          reinterpret_cast<uint4*>(xs)[((g * 4 + jq) * M + m) * 4 + cq] = v;
-        if (kOffset) {
-          const float2 lx = act2_to_float2<kBf16>(v.x), hy = act2_to_float2<kBf16>(v.y);
-          const float2 lz = act2_to_float2<kBf16>(v.z), hw = act2_to_float2<kBf16>(v.w);
-          const float lo = (lx.x + lx.y) + (lz.x + lz.y), hi = (hy.x + hy.y) + (hw.x + hw.y);
-          c1 += lo + hi;
-          c2 += kDiv16 ? lo + 16.0f * hi : lo + hi;
+      for (int e = 0; e < kG4XRound; ++e) {
+        if (base + e * kG4Warps * 32 >= nch) break;
+        const int i = base + e * kG4Warps * 32 + tid;
+        v[e] = i < nch ? *reinterpret_cast<const uint4*>(X + static_cast<int64_t>(i) * 8)
+                       : make_uint4(0u, 0u, 0u, 0u);
+        if (inv_s != nullptr && i < nch) {
+          const int k = (i % kpr) * 8;
+          s0[e] = *reinterpret_cast<const float4*>(inv_s + k);
+          s1[e] = *reinterpret_cast<const float4*>(inv_s + k + 4);
         }
       }
-      if (kOffset) {
 #pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
-          c1 += __shfl_xor_sync(0xffffffffu, c1, o);
-          c2 += __shfl_xor_sync(0xffffffffu, c2, o);
+      for (int e = 0; e < kG4XRound; ++e) {
+        if (base + e * kG4Warps * 32 >= nch) break;   // the same for every thread
+        const int i = base + e * kG4Warps * 32 + tid;
+        const bool live = i < nch;   // whole 16-lane blocks are live or not
+        const int m = i / kpr, rem = i % kpr, g = rem >> 4, ch = rem & 15;
+        if (inv_s != nullptr && live) v[e] = scale8<kBf16>(v[e], s0[e], s1[e]);
+        if (kOffset && kDiv16) {
+          v[e].y = h2_as_u32(__hmul2(u32_as_h2(v[e].y), sixteenth));
+          v[e].w = h2_as_u32(__hmul2(u32_as_h2(v[e].w), sixteenth));
         }
-        if (sub == 0 && live) {
-          // C1 = base * sum of the staged values (c1 == c2 unless kDiv16)
-          cc[(g * kTok + m) * 2] = kBf16 ? 128.0f * c2 : 1024.0f * c1;
-          cc[(g * kTok + m) * 2 + 1] = c2;
+        // chunk ch holds k = 8 ch .. 8 ch + 7 of the group: 32-k quarter ch / 4, 8-k chunk ch % 4
+        const int dst = ((g * 4 + (ch & 3)) * M + m) * 4 + (ch >> 2);
+        if (live && AWQ_IN_BOUNDS(dst < G * 16 * M)) reinterpret_cast<uint4*>(xs)[dst] = v[e];
+        if (kOffset) {
+          const float2 lx = act2_to_float2<kBf16>(v[e].x), hy = act2_to_float2<kBf16>(v[e].y);
+          const float2 lz = act2_to_float2<kBf16>(v[e].z), hw = act2_to_float2<kBf16>(v[e].w);
+          const float lo = (lx.x + lx.y) + (lz.x + lz.y), hi = (hy.x + hy.y) + (hw.x + hw.y);
+          float c1 = lo + hi, c2 = kDiv16 ? lo + 16.0f * hi : lo + hi;
+#pragma unroll
+          for (int o = 1; o < 16; o <<= 1) {
+            c1 += __shfl_xor_sync(0xffffffffu, c1, o);
+            c2 += __shfl_xor_sync(0xffffffffu, c2, o);
+          }
+          if (ch == 0 && live) {
+            // C1 = base * sum of the staged values (c1 == c2 unless kDiv16)
+            cc[(g * kTok + m) * 2] = kBf16 ? 128.0f * c2 : 1024.0f * c1;
+            cc[(g * kTok + m) * 2 + 1] = c2;
+          }
         }
       }
     }
     if (kOffset)
-      for (int i = threadIdx.x; i < G * kTok; i += kG4Warps * 32)
-        if (i % kTok >= M) { cc[2 * i] = 0.0f; cc[2 * i + 1] = 0.0f; }
+      for (int i = tid; i < G * kTok; i += kG4Warps * 32)
+        if (i % kTok >= M) {
+          cc[2 * i] = 0.0f;
+          cc[2 * i + 1] = 0.0f;
+        }
     named_bar_sync(1, kG4Warps * 32);
   }
 
