@@ -89,6 +89,18 @@ def profiled_traffic(kernel):
     return None, ("kernel changed since its ncu capture" if seen else "no ncu capture")
 
 
+def search_executed_flops(M, N, K, n_alpha):
+    """Tensor-core flops one awq_search_scale call executes, and its form. Direct (M < 2K):
+    both fp16 parts of the error operand times X, 2 * n_alpha * 2 M N_pad K. Gram (M >= 2K):
+    G = X^T X once over the token-padded X (2 M_pad K^2), then three MMAs per k step (hi*hi,
+    hi*lo, lo*hi) of the error operand against G, n_alpha * 3 * 2 N_pad K^2."""
+    n_pad = -(-N // 128) * 128
+    if M >= 2 * K:
+        m_pad = -(-M // 128) * 128
+        return 2 * m_pad * K * K + n_alpha * 3 * 2 * n_pad * K * K, "gram"
+    return 2 * n_alpha * 2 * M * n_pad * K, "direct"
+
+
 def gemm_bytes(M, N, K, bits=4):
     return N * K * bits // 8 + N * (K // GROUP) * 3 + 2 * M * K + 2 * M * N
 
@@ -355,11 +367,12 @@ def decoder_layer_rows(awq, dev, pk):
                      device=dev)
     t = time_call(lambda: awq.awq_search_scale(Wgu, X, sx, alphas, 4, workspace=ws), 2)
     flops = 20 * 2 * M * Ngu * K
-    # the error operand's two fp16 parts each go through the tensor cores: 2x the MMA work
+    ex, form = search_executed_flops(M, Ngu, K, 20)
     rows["search_gate_up"] = {"M": M, "N": Ngu, "K": K, "grid": 20, "ms": t * 1e3,
-                              "TFLOP/s (algorithmic 20*2MNK)": flops / t / 1e12,
-                              "TFLOP/s (executed, two-part operand)": 2 * flops / t / 1e12,
-                              "frac_tensor_executed": 2 * flops / t / 1e12 / pk["bf16_tflops"]}
+                              "form": form,
+                              "TFLOP/s (definition, 20*2MNK)": flops / t / 1e12,
+                              "TFLOP/s (executed)": ex / t / 1e12,
+                              "frac_tensor_executed": ex / t / 1e12 / pk["bf16_tflops"]}
     del ws, Wgu
     torch.cuda.empty_cache()
 
@@ -391,7 +404,7 @@ def decoder_layer_rows(awq, dev, pk):
         W = stacked[tuple(names)]
         _, best, best_s, _, best_inv = awq.awq_search_scale(W, Xd[xname], stats[xname], alphas,
                                                             4, workspace=search_ws, inv=True)
-        search_flops += 20 * 2 * Xd[xname].shape[0] * W.shape[0] * W.shape[1]
+        search_flops += search_executed_flops(Xd[xname].shape[0], W.shape[0], W.shape[1], 20)[0]
         for n in names:
             chosen[n] = (best, best_s, best_inv)
     ev[2].record()
@@ -415,7 +428,7 @@ def decoder_layer_rows(awq, dev, pk):
     rows["decoder_layer_pipeline"] = {
         "tokens": int(Xd["hidden"].shape[0]), "seconds": sum(st),
         "stats_and_gated_input_s": st[0], "search_s": st[1], "pack_s": st[2], "gemm_s": st[3],
-        "search_TFLOP/s": search_flops / st[1] / 1e12,
+        "search_TFLOP/s (executed)": search_flops / st[1] / 1e12,
         "gemm_TFLOP/s": gemm_flops / st_gemm_only / 1e12,
         "alpha_index": {n: int(chosen[n][0].item()) for n in chosen},
     }
@@ -702,7 +715,7 @@ def run_b200(args, world, rank, local):
                      "unit": "GB/s", "frac": per_gpu / pk["hbm_gbs"],
                      "traffic": dec_traffic, "traffic_source": dec_traffic_src,
                      "algorithmic_bytes_per_launch": step_bytes / len(synth.DECODE_SHAPES),
-                     "kernel": "gemv_stream_kernel<1, true, 8>", "peak_source": pk["source"],
+                     "kernel": "gemv_stream_kernel<1, true, false, 4>", "peak_source": pk["source"],
                      "peak_kind": "measured copy bandwidth (burst)",
                      "frac_of_8TBps_nominal": per_gpu / 8000.0},
         "prefill": {"metric": "TFLOP/s at M=2048", "value": pf_value, "unit": "TFLOP/s",

@@ -219,6 +219,30 @@ def test_gemm_split_k_ragged(awq, M, N, K, bits):
     _check_gemm(awq, X, qw, sc, z, N, K, bits)
 
 
+def test_gemm_split_k_ragged_large_is_linear_time(awq):
+    # M * N = 33 * 4097 is odd and the output has few 128-row tiles, so the split-K partials
+    # go through the reduction's ragged tail. A reduction whose tail loop ran over the whole
+    # remaining output per thread (quadratic work) takes seconds here; the correct one
+    # takes microseconds. Checked against the oracle, then timed after a warm-up.
+    M, N, K = 33, 4097, 4096
+    W, X, m = rand_layer(M + N + K, N, K, M)
+    qw, sc, z = _packed(W, np.sqrt(m).astype(np.float32))
+    _check_gemm(awq, X, qw, sc, z, N, K)
+    Xd, q, s_, zd = cu(X), cu(qw), cu(sc), cu(z)
+    Y = torch.empty(M, N, dtype=torch.float16, device="cuda")
+    for _ in range(3):
+        awq.awq_gemm_w4a16(Xd, q, s_, zd, N, K, 4, out=Y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(10):
+        awq.awq_gemm_w4a16(Xd, q, s_, zd, N, K, 4, out=Y)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / 10
+    assert ms < 1.0, f"{ms:.3f} ms per call"
+
+
 @pytest.mark.parametrize("bits", [4, 3])
 @pytest.mark.parametrize("M,N,K", [(40, 512, 2304), (20, 640, 1152), (96, 256, 1664),
                                    (250, 384, 640)])
