@@ -92,12 +92,15 @@ def profiled_traffic(kernel):
 def search_executed_flops(M, N, K, n_alpha):
     """Tensor-core flops one awq_search_scale call executes, and its form. Direct (M < 2K):
     both fp16 parts of the error operand times X, 2 * n_alpha * 2 M N_pad K. Gram (M >= 2K):
-    G = X^T X once over the token-padded X (2 M_pad K^2), then three MMAs per k step (hi*hi,
-    hi*lo, lo*hi) of the error operand against G, n_alpha * 3 * 2 N_pad K^2."""
+    the tiles of G = X^T X on or above the diagonal over the token-padded X (about M_pad K^2),
+    then three MMAs per k step (hi*hi, hi*lo, lo*hi) of the error operand against G,
+    n_alpha * 3 * 2 N_pad K^2."""
     n_pad = -(-N // 128) * 128
     if M >= 2 * K:
         m_pad = -(-M // 128) * 128
-        return 2 * m_pad * K * K + n_alpha * 3 * 2 * n_pad * K * K, "gram"
+        # G is built from its 128 x 256 tiles that reach the diagonal or above it
+        tiles = sum(1 for r in range(K // 128) for c in range(-(-K // 256)) if r * 128 < (c + 1) * 256)
+        return 2 * m_pad * 128 * 256 * tiles + n_alpha * 3 * 2 * n_pad * K * K, "gram"
     return 2 * n_alpha * 2 * M * n_pad * K, "direct"
 
 

@@ -604,6 +604,7 @@ awq_status awq_search_scale(const awq_f16* W, int64_t N, int64_t K, const awq_f1
     ga.N_pad = K;
     ga.K = lay.M_pad;    // the contraction runs over tokens
     ga.G = G;
+    ga.upper_only = 1;   // G is symmetric: the tiles at or above the diagonal suffice
     // the contraction over tokens in slices of about 2048 (128 accumulation steps each)
     ga.k_splits = static_cast<int>(lay.M_pad / 2048 > 1 ? lay.M_pad / 2048 : 1);
     s = launch_tc<256, ASrc::kFp16x1, Epi::kStoreF32>(XT, K, XT, K, ga, st);

@@ -133,6 +133,8 @@ struct TcArgs {
                         // (needs N % 16 == 0); else the builders load them from global memory
   const float* inv_s;   // packed source: NULL, or [K] factors folded into the weights
   float* G;             // kStoreF32: [rows_total, M] fp32 output (the Gram matrix)
+  int upper_only;       // kStoreF32: compute only the tiles that reach the diagonal or above it
+                        // (G is symmetric; readers take G[min(i,j)][max(i,j)])
   const __half* E2;     // kGramDot: the error operand [rows_total, 2K] the epilogue reads
 };
 
@@ -281,6 +283,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int lane = threadIdx.x & 31;
   const int64_t units =
       static_cast<int64_t>(args.row_tiles) * args.m_tiles * args.k_splits;
+  if (kEpi == Epi::kStoreF32 && args.upper_only) {
+    // One CTA per output tile: a tile whose rows all lie below its columns (every element
+    // G[i][j] with i > j) is the transpose of a computed one, so its CTA has nothing to do.
+    int row_tile, m_tile;
+    tile_of_block(blockIdx.x % (static_cast<int64_t>(args.row_tiles) * args.m_tiles),
+                  args.row_tiles, args.m_tiles, row_tile, m_tile);
+    if (static_cast<int64_t>(row_tile) * kTcBM >= static_cast<int64_t>(m_tile + 1) * BN) return;
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {

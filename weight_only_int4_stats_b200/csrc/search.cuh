@@ -112,14 +112,17 @@ __global__ void gram_rms_kernel(const float* __restrict__ G, int64_t K, int64_t 
 
 // G2[i] = [hi | lo] of G'[i][j] = G[i][j] / (sqrt(G[i][i]) sqrt(G[j][j])) (0 when either
 // channel is dead): hi = fp16(g'), lo = fp16((g' - hi) * 2^12), as for the error operand.
+// Only the tiles of G on or above the diagonal are computed; G[i][j] is read as
+// G[min(i,j)][max(i,j)], so G' is exactly symmetric.
 __global__ void gram_normalize_kernel(const float* __restrict__ G, int64_t K,
                                       __half* __restrict__ G2) {
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t i = blockIdx.y;
   if (j >= K) return;
   const float gii = G[i * K + i], gjj = G[j * K + j];
+  const int64_t lo = i < j ? i : j, hi_ = i < j ? j : i;
   float g = 0.0f;
-  if (gii > 0.0f && gjj > 0.0f) g = G[i * K + j] / (sqrtf(gii) * sqrtf(gjj));
+  if (gii > 0.0f && gjj > 0.0f) g = G[lo * K + hi_] / (sqrtf(gii) * sqrtf(gjj));
   const __half hi = __float2half_rn(g);
   G2[i * 2 * K + j] = hi;
   G2[i * 2 * K + K + j] = __float2half_rn(__fmul_rn(__fsub_rn(g, __half2float(hi)), 4096.0f));
