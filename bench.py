@@ -475,6 +475,81 @@ def profile_rows(awq, dev):
     torch.cuda.synchronize()
 
 
+def trace_decode(awq, dev, l2, stream, steps):
+    """The headline step (M = 1 on the three decode shapes, weights-ready, one CUDA graph) on
+    the trace build: the per-launch timeline of the streaming decode kernel from its CTAs'
+    %globaltimer records. Steady-state medians per shape, in microseconds:
+      span: from the previous launch's last CTA end to this launch's last CTA end;
+      early_start: how long before the previous launch ended this launch's first CTA started;
+      wait_release: from the previous launch's end to this launch's dependency wait returning
+        (the producer's; mean over CTAs);
+      x_staging: from that wait to X staged in shared memory (mean over CTAs; the consumers'
+        own wait may return before the producer's);
+      per_unit: interval between consecutive units (16 KB of codes) landing (mean over CTAs);
+      units_max: the most units any CTA of the launch has;
+      tail: from the mean CTA end to the last CTA end.
+    %globaltimer ticks every 256 ns on this part; the means over CTAs and steps resolve below
+    that."""
+    from weight_only_int4_stats_b200 import build
+    awq.use_library(build.build(trace=True))
+    shapes = [DecodeShape(awq, N, K, 1, l2, dev) for (N, K) in synth.DECODE_SHAPES]
+    for sh in shapes:
+        sh.call(awq, 1, 0)
+    torch.cuda.synchronize()
+    g = capture_run(lambda r: [sh.call(awq, 1, r) for sh in shapes], 0, steps, stream)
+    with torch.cuda.stream(stream):
+        g.replay()            # the first replay uploads the graph
+    torch.cuda.synchronize()
+    awq.trace_reset()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    step_us = e0.elapsed_time(e1) * 1e3 / steps
+    R = awq.trace_read().astype(np.int64)
+    # a launch's CTAs all start before the next launch's first CTA (which launches only after
+    # every CTA of this one has passed its dependency wait); each blockIdx appears once
+    launches, cur, seen = [], [], set()
+    for rec in R:
+        b = int(rec[6])
+        if b in seen:
+            launches.append(np.array(cur))
+            cur, seen = [], set()
+        cur.append(rec)
+        seen.add(b)
+    if cur:
+        launches.append(np.array(cur))
+    per = {j: [] for j in range(len(shapes))}
+    for li in range(len(shapes), len(launches)):
+        L, prev = launches[li], launches[li - 1]
+        j = li % len(shapes)
+        prev_end = prev[:, 5].max()
+        units = L[:, 1]
+        gaps = []
+        for rec, n in zip(L, units):
+            k = int(min(n, 24))
+            if k >= 2:   # first-to-last over k - 1 intervals
+                gaps.append((rec[8 + k - 1] - rec[8]) / (k - 1))
+        # %globaltimer ticks coarsely (256 ns here): means over the CTAs average the tick out
+        per[j].append([L[:, 5].max() - prev_end, prev_end - L[:, 2].min(),
+                       L[:, 3].mean() - prev_end, (L[:, 4] - L[:, 3]).mean(),
+                       np.mean(gaps) if gaps else float("nan"), units.max(),
+                       L[:, 5].max() - L[:, 5].mean()])
+    keys = ["span", "early_start", "wait_release", "x_staging", "per_unit", "units_max", "tail"]
+    out = []
+    for j, sh in enumerate(shapes):
+        m = np.median(np.array(per[j], dtype=np.float64), axis=0)
+        row = {"N": sh.N, "K": sh.K}
+        for k, v in zip(keys, m):
+            row[k] = int(v) if k == "units_max" else round(float(v) / 1e3, 3)
+        out.append(row)
+    print(json.dumps({"metric": "decode timeline (trace build), M=1", "steps": steps,
+                      "step_us": round(step_us, 2), "launches": len(launches),
+                      "per_shape": out}), flush=True)
+
+
 # ----------------------------------------------------------------------------- main arms
 
 def run_reference(args, world, rank):
@@ -528,6 +603,9 @@ def run_b200(args, world, rank, local):
     stream = torch.cuda.Stream()
     if args.only == "profile":
         profile_rows(awq, dev)
+        return
+    if args.only == "trace":
+        trace_decode(awq, dev, l2, stream, args.steps)
         return
     if args.only == "rows":
         rows = decoder_layer_rows(awq, dev, pk)
@@ -747,7 +825,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--only", choices=["all", "decode", "batched", "prefill", "bf16", "rows",
-                                       "profile"],
+                                       "profile", "trace"],
                     default="all",
                     help="run one section only (used by the profiling commands)")
     args = ap.parse_args()

@@ -95,6 +95,23 @@ AWQ_API awq_status awq_selftest_timeout(int* waited_out, void* stream);
  * The release build has no checks and returns AWQ_ERR_UNSUPPORTED without launching. */
 AWQ_API awq_status awq_selftest_bounds(int* buf, void* stream);
 
+/* Timeline of the trace build (libawq_b200_trace.so, compiled with AWQ_TRACE). In that build
+ * the streaming decode kernel (awq_gemm_w4a16 with M <= 16 on its default path) records
+ * %globaltimer nanoseconds at fixed points of every CTA: one record of AWQ_TRACE_WORDS
+ * 64-bit words per CTA, in the order the CTAs start, for up to 65536 CTAs after the last
+ * reset. Record words: 0 N of the launch; 1 units (tile, 2048-k chunk) of the CTA; 2 CTA
+ * start; 3 the dependency wait returned (griddepcontrol.wait: the preceding kernel on the
+ * stream has completed); 4 X staged in shared memory; 5 the CTA's last unit done;
+ * 6 blockIdx.x; 8 + u (u < 24) unit u's packed weights have landed in shared memory and
+ * the consumers start on it.
+ * awq_trace_reset: synchronous; clears the record count.
+ * awq_trace_read: synchronous; copies min(count, max_ctas) records to host memory `out`
+ * (max_ctas * AWQ_TRACE_WORDS words, caller-owned) and the record count to *n_ctas.
+ * The release and debug builds record nothing and return AWQ_ERR_UNSUPPORTED. */
+#define AWQ_TRACE_WORDS 32
+AWQ_API awq_status awq_trace_reset(void);
+AWQ_API awq_status awq_trace_read(unsigned long long* out, int64_t max_ctas, int64_t* n_ctas);
+
 /* ---------------------------------------------------------------- activation statistics
  * robotsatlas.com "AWQ", "How it works" / "Components: Activation saliency analysis":
  * the activation magnitude of every input channel on the calibration set,

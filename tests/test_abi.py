@@ -140,3 +140,20 @@ def test_debug_build_exports_the_same_symbols():
     assert D.awq_abi_version() == 2
     # the release build refuses the bounds self-test without launching anything
     assert _lib().awq_selftest_bounds(ctypes.c_void_p(1 << 20), None) == 2
+
+
+def test_trace_build_exports_the_same_symbols():
+    # the timeline build is the same library with %globaltimer stamps in the decode kernel;
+    # the release and debug builds decline the trace calls without touching the GPU
+    from weight_only_int4_stats_b200 import build
+    import weight_only_int4_stats_b200 as awq
+    T = awq.load_library(build.build(trace=True))
+    for name in _declared():
+        assert hasattr(T, name), name
+    assert T.awq_abi_version() == 2
+    n = ctypes.c_int64(0)
+    out = (ctypes.c_ulonglong * 32)()
+    assert _lib().awq_trace_reset() == 2
+    assert _lib().awq_trace_read(out, 1, ctypes.byref(n)) == 2
+    D = awq.load_library(build.build(debug=True))
+    assert D.awq_trace_reset() == 2

@@ -52,6 +52,8 @@ def load_library(path: str) -> ctypes.CDLL:
         "awq_check_error": (I32, [P]),
         "awq_selftest_timeout": (I32, [P, P]),
         "awq_selftest_bounds": (I32, [P, P]),
+        "awq_trace_reset": (I32, []),
+        "awq_trace_read": (I32, [P, I64, P]),
         "awq_act_stats_workspace_size": (SZ, [I64, I64]),
         "awq_act_stats": (I32, [P, I64, I64, P, P, SZ, P]),
         "awq_act_stats_noalloc": (I32, [P, I64, I64, P, P]),
@@ -77,6 +79,32 @@ def lib() -> ctypes.CDLL:
     if _lib is None:
         _lib = load_library(library_path)
     return _lib
+
+
+def use_library(path: str) -> ctypes.CDLL:
+    """Makes the build at `path` (e.g. the trace build) the one every call of this module
+    goes through, and returns it."""
+    global _lib
+    _lib = load_library(path)
+    return _lib
+
+
+def trace_read(max_ctas: int = 1 << 16):
+    """The trace build's per-CTA timeline records since the last awq_trace_reset, as a
+    [n, AWQ_TRACE_WORDS] uint64 numpy array (see include/awq.h). Raises AwqError with
+    AWQ_ERR_UNSUPPORTED on a build without the timeline."""
+    import numpy as np
+    words = 32
+    out = np.zeros((max_ctas, words), dtype=np.uint64)
+    n = ctypes.c_int64(0)
+    _check("awq_trace_read", lib().awq_trace_read(ctypes.c_void_p(out.ctypes.data), max_ctas,
+                                                  ctypes.byref(n)))
+    return out[:min(n.value, max_ctas)]
+
+
+def trace_reset():
+    """Clears the trace build's timeline records."""
+    _check("awq_trace_reset", lib().awq_trace_reset())
 
 
 def _ptr(t):

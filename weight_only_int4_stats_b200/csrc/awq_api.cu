@@ -365,6 +365,41 @@ awq_status awq_selftest_bounds(int* buf, void* stream) {
 #endif
 }
 
+awq_status awq_trace_reset(void) {
+#ifdef AWQ_TRACE
+  static_assert(awq::kTraceWords == AWQ_TRACE_WORDS, "trace record size");
+  const unsigned zero = 0;
+  if (cudaMemcpyToSymbol(awq::g_trace_ctas, &zero, sizeof(zero)) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  return AWQ_OK;
+#else
+  return AWQ_ERR_UNSUPPORTED;   // only the trace build records a timeline
+#endif
+}
+
+awq_status awq_trace_read(unsigned long long* out, int64_t max_ctas, int64_t* n_ctas) {
+#ifdef AWQ_TRACE
+  if (out == nullptr || n_ctas == nullptr || max_ctas < 0) return AWQ_ERR_INVALID_ARG;
+  unsigned count = 0;
+  if (cudaMemcpyFromSymbol(&count, awq::g_trace_ctas, sizeof(count)) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  int64_t n = count < static_cast<unsigned>(awq::kTraceCtas) ? count : awq::kTraceCtas;
+  if (n > max_ctas) n = max_ctas;
+  if (n > 0 &&
+      cudaMemcpyFromSymbol(out, awq::g_trace,
+                           static_cast<size_t>(n) * awq::kTraceWords * sizeof(unsigned long long)) !=
+          cudaSuccess)
+    return AWQ_ERR_CUDA;
+  *n_ctas = count;
+  return AWQ_OK;
+#else
+  (void)out;
+  (void)max_ctas;
+  (void)n_ctas;
+  return AWQ_ERR_UNSUPPORTED;
+#endif
+}
+
 awq_status awq_selftest_timeout(int* waited_out, void* stream) {
   if (waited_out == nullptr || (reinterpret_cast<uintptr_t>(waited_out) & 3u) != 0)
     return AWQ_ERR_INVALID_ARG;

@@ -48,6 +48,37 @@ __device__ __forceinline__ bool bounds_ok(bool cond) {
 #define AWQ_IN_BOUNDS(cond) (true)
 #endif
 
+// Timeline of the trace build (compiled with AWQ_TRACE): the streaming decode kernel records
+// %globaltimer at fixed points of each CTA into g_trace, one record of kTraceWords words per
+// CTA in the order the CTAs start (g_trace_ctas counts them; records past kTraceCtas are
+// dropped). In the release and debug builds AWQ_TRACE_AT compiles away.
+constexpr int kTraceWords = 32;
+constexpr int kTraceCtas = 1 << 16;
+// Record layout (word: content)
+constexpr int kTrN = 0;          // N of the launch
+constexpr int kTrUnits = 1;      // units of this CTA
+constexpr int kTrStart = 2;      // CTA start
+constexpr int kTrWaited = 3;     // the producer's griddepcontrol.wait returned
+constexpr int kTrXStaged = 4;    // X staged in shared memory (consumers' barrier passed)
+constexpr int kTrEnd = 5;        // the consumers' last unit done
+constexpr int kTrBlock = 6;      // blockIdx.x
+constexpr int kTrUnit0 = 8;      // 8 + u: consumer warp 0 saw unit u land (u < 24)
+constexpr int kTrMaxUnits = kTraceWords - kTrUnit0;
+#ifdef AWQ_TRACE
+__device__ unsigned long long g_trace[static_cast<size_t>(kTraceCtas) * kTraceWords];
+__device__ unsigned int g_trace_ctas;
+#define AWQ_TRACE_AT(rec, word, value)                                                        \
+  do {                                                                                       \
+    if ((rec) < static_cast<unsigned>(::awq::kTraceCtas))                                    \
+      ::awq::g_trace[static_cast<size_t>(rec) * ::awq::kTraceWords + (word)] =               \
+          static_cast<unsigned long long>(value);                                            \
+  } while (0)
+#else
+#define AWQ_TRACE_AT(rec, word, value) \
+  do {                                 \
+  } while (0)
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

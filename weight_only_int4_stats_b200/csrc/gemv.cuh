@@ -376,14 +376,30 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
   const int C = (Ki + kG4KC - 1) / kG4KC;
   const int64_t units = (t1 - t0) * C;
 
+  // the trace build's record index of this CTA lives in the barrier area's spare word
+  unsigned* trace_rec = reinterpret_cast<unsigned*>(empty + kGSMaxSlots);
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kG4Warps * 32);
     }
     fence_barrier_init();
+#ifdef AWQ_TRACE
+    *trace_rec = atomicAdd(&g_trace_ctas, 1u);
+    AWQ_TRACE_AT(*trace_rec, kTrStart, globaltimer_ns());
+    AWQ_TRACE_AT(*trace_rec, kTrN, N);
+    AWQ_TRACE_AT(*trace_rec, kTrUnits, units);
+    AWQ_TRACE_AT(*trace_rec, kTrBlock, blockIdx.x);
+#endif
   }
   __syncthreads();
+#ifdef AWQ_TRACE
+  const unsigned rec = *trace_rec;
+#else
+  const unsigned rec = 0u;
+  (void)trace_rec;
+#endif
+  (void)rec;
 
   if (warp == kG4Warps) {
     // ---------------------------------------------------------------- producer
@@ -423,6 +439,7 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
           prefetch_l2_bulk(wrow + off, static_cast<uint32_t>(bytes - off < 65536 ? bytes - off : 65536));
       }
       pdl_wait();
+      AWQ_TRACE_AT(rec, kTrWaited, globaltimer_ns());
       // every kernel before this one has completed: the next grid may now be scheduled
       pdl_launch_dependents();
       for (; u < units; ++u) {
@@ -501,6 +518,7 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
           cc[2 * i + 1] = 0.0f;
         }
     named_bar_sync(1, kG4Warps * 32);
+    if (threadIdx.x == 0) AWQ_TRACE_AT(rec, kTrXStaged, globaltimer_ns());
   }
 
   // A timed-out wait clears `ok`; the warp then skips further waits and arithmetic but still
@@ -517,6 +535,7 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
   int64_t tile = t0;
   for (int64_t u = 0; u < units; ++u) {
     ok = __all_sync(0xffffffffu, ok && mbar_wait(&full[slot], ph));
+    if (threadIdx.x == 0 && u < kTrMaxUnits) AWQ_TRACE_AT(rec, kTrUnit0 + u, globaltimer_ns());
     // Copy this warp's operands of the unit (its two groups: packed codes of rows r and r + 8,
     // their scales and zero points) to registers and release the slot at once, so the
     // producer refills it while this unit is computed. Every lane arrives (release
@@ -678,6 +697,7 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
     }
     if (++chunk == C) { chunk = 0; ++tile; }
   }
+  if (threadIdx.x == 0) AWQ_TRACE_AT(rec, kTrEnd, globaltimer_ns());
 }
 
 }  // namespace awq
