@@ -225,7 +225,8 @@ namespace awq {
 // an SM's shared memory, so the next GEMM's CTAs become resident beside this one's as soon as
 // every CTA of this grid has passed griddepcontrol.wait (where the next launch is allowed).
 // Before the wait a CTA touches no output and no activation: it issues L2 prefetches of its
-// weight rows (coherent with writes of the preceding kernel, so always safe) and, when the
+// weight rows, of X and of inv_s (coherent with writes of the preceding kernel, so always
+// safe) and, when the
 // caller states that the weights are not written by the kernel launched just before
 // (kGemvWeightsReady), TMA-loads the first ring slots.
 //
@@ -437,6 +438,16 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
         const int64_t bytes = (r1 - r0) * row_bytes;
         for (int64_t off = 0; off < bytes; off += 65536)
           prefetch_l2_bulk(wrow + off, static_cast<uint32_t>(bytes - off < 65536 ? bytes - off : 65536));
+        // X and inv_s too: an L2 prefetch is coherent with the preceding kernel's writes
+        // (L2 is where they land), and the staging loads after the wait then hit L2
+        const int64_t xb = static_cast<int64_t>(M) * K * 2;
+        for (int64_t off = 0; off < xb; off += 65536)
+          prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(X) + off,
+                           static_cast<uint32_t>(xb - off < 65536 ? xb - off : 65536));
+        if (inv_s != nullptr)
+          for (int64_t off = 0; off < K * 4; off += 65536)
+            prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(inv_s) + off,
+                             static_cast<uint32_t>(K * 4 - off < 65536 ? K * 4 - off : 65536));
       }
       pdl_wait();
       AWQ_TRACE_AT(rec, kTrWaited, globaltimer_ns());
@@ -474,7 +485,7 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
         v[e] = i < nch ? *reinterpret_cast<const uint4*>(X + static_cast<int64_t>(i) * 8)
                        : make_uint4(0u, 0u, 0u, 0u);
         if (inv_s != nullptr && i < nch) {
-          const int k = (i % kpr) * 8;
+          const int k = (M == 1 ? i : i % kpr) * 8;
           s0[e] = *reinterpret_cast<const float4*>(inv_s + k);
           s1[e] = *reinterpret_cast<const float4*>(inv_s + k + 4);
         }
@@ -484,7 +495,8 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
         if (base + e * kG4Warps * 32 >= nch) break;   // the same for every thread
         const int i = base + e * kG4Warps * 32 + tid;
         const bool live = i < nch;   // whole 16-lane blocks are live or not
-        const int m = i / kpr, rem = i % kpr, g = rem >> 4, ch = rem & 15;
+        // (M = 1: one token row, no division)
+        const int m = M == 1 ? 0 : i / kpr, rem = M == 1 ? i : i % kpr, g = rem >> 4, ch = rem & 15;
         if (inv_s != nullptr && live) v[e] = scale8<kBf16>(v[e], s0[e], s1[e]);
         if (kOffset && kDiv16) {
           v[e].y = h2_as_u32(__hmul2(u32_as_h2(v[e].y), sixteenth));
