@@ -93,10 +93,14 @@ struct TcLayout {
   static constexpr int kPBytes = kTcBM * kPRowBytes;
   // the slot's fp16 scales [kPG][128] then its zero points [kPG][128]
   static constexpr int kSZBytes = kPG * (kTcBM * 2 + kTcBM);
+  // the slot's inv_s [kPG][128] fp32 (packed sources with inv_s): the builders read it from
+  // shared memory, broadcast across the tile's rows
+  static constexpr int kInvBytes = kPk ? kPG * kGroup * 4 : 0;
   // as many packed slots as the shared memory left by the stages holds (1024 bytes of
   // alignment slack and 512 of barriers reserved)
   static constexpr int kPFit =
-      (kTcSmemMax - 1024 - 512 - kStages * (kXBytes + kABytes)) / (kPBytes + kSZBytes);
+      (kTcSmemMax - 1024 - 512 - kStages * (kXBytes + kABytes)) /
+      (kPBytes + kSZBytes + kInvBytes);
   static constexpr int kPSlots =
       !kPk ? 0 : (kPFit < kTcPkSlotsMax ? kPFit : kTcPkSlotsMax);
   static constexpr int kPBars = kPSlots > 0 ? kPSlots : 1;   // barrier pairs of the ring
@@ -104,7 +108,8 @@ struct TcLayout {
   static constexpr int kAOff = kXOff + kStages * kXBytes;
   static constexpr int kPOff = kAOff + kStages * kABytes;
   static constexpr int kSZOff = kPOff + kPSlots * kPBytes;
-  static constexpr int kBarOff = kSZOff + kPSlots * kSZBytes;
+  static constexpr int kIOff = kSZOff + kPSlots * kSZBytes;
+  static constexpr int kBarOff = kIOff + kPSlots * kInvBytes;
   // full[S], empty[S], built[S], pfull[P], pempty[P], acc_full[2], acc_empty[2], tmem slot
   static constexpr int kBytes = kBarOff + (3 * kStages + 2 * kPBars + 4) * 8 + 16;
   static constexpr int kSmem = kBytes + 1024;   // slack for 1024-byte alignment
@@ -191,7 +196,8 @@ __device__ __forceinline__ uint4 dequant_word_scaled(uint32_t w, __half2 bias_lo
 }
 
 // The four scale pairs of 8 consecutive k starting at k0: fp16(sc * inv_s[k]) pairs, or sc
-// broadcast when inv_s is NULL (bf16 pairs for bf16 activations). Folding inv_s into the
+// broadcast when inv_s is NULL (bf16 pairs for bf16 activations). inv_s points at the
+// group's factors in the packed slot (shared memory) and k0 is relative to the group. Folding inv_s into the
 // weights computes sum_k x[k] * (inv_s[k] * deq[k]) = sum_k (x[k] * inv_s[k]) * deq[k].
 template <bool kBf16 = false>
 __device__ __forceinline__ uint4 pair_scales(float sc, uint32_t sc2, const float* inv_s,
@@ -469,6 +475,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t sc = kBf16 ? float2_to_act2<true>(scf, scf) : h2_as_u32(__half2half2(sv));
           const uint32_t bias = kBf16 ? (0x4300u | z) * 0x00010001u : h2_as_u32(lo);
           const uint8_t* prow = smem + L::kPOff + ps * L::kPBytes + r * L::kPRowBytes;
+          // this group's inv_s in the slot (k relative to the group), or NULL
+          const float* inv_g =
+              args.inv_s == nullptr
+                  ? nullptr
+                  : reinterpret_cast<const float*>(smem + L::kIOff + ps * L::kInvBytes) +
+                        gi * kGroup;
 #pragma unroll
           for (int e = 0; e < 2; ++e) {             // stage i + e of the group
             uint8_t* atile = smem + L::kAOff + (e ? s1 : s) * L::kABytes;
@@ -478,8 +490,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                const int64_t k0 = static_cast<int64_t>(kb + e) * kTcBK + 32 * h + 8 * q;
-                const uint4 c4 = pair_scales<kBf16>(scf, sc, args.inv_s, k0);
+                const int k0 = e * kTcBK + 32 * h + 8 * q;   // k inside the group
+                const uint4 c4 = pair_scales<kBf16>(scf, sc, inv_g, k0);
                 const uint4 o = kBf16 ? dequant_word_scaled_bf16(words[q], bias, c4)
                                       : dequant_word_scaled(words[q], lo, hi, c4);
                 *reinterpret_cast<uint4*>(atile + sw128_offset(r, 4 * h + q)) = o;
@@ -490,8 +502,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const uint32_t w0 = pw[0], w1 = pw[1], w2 = pw[2];
               uint4 o, c4;
 #define AWQ_DQ3_CHUNK(I)                                                                    \
-  c4 = pair_scales<kBf16>(scf, sc, args.inv_s,                                             \
-                          static_cast<int64_t>(kb + e) * kTcBK + 32 * h + 8 * (I));        \
+  c4 = pair_scales<kBf16>(scf, sc, inv_g, e * kTcBK + 32 * h + 8 * (I));                  \
   o.x = dequant3_pair<I, 0, kBf16>(w0, w1, w2, bias, c4.x);                                \
   o.y = dequant3_pair<I, 1, kBf16>(w0, w1, w2, bias, c4.y);                                \
   o.z = dequant3_pair<I, 2, kBf16>(w0, w1, w2, bias, c4.z);                                \
@@ -654,9 +665,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&pfull[ps], L::kPBytes + (args.sz_tma ? L::kSZBytes : 0));
+          // inv_s of the slot's groups that lie inside K (a bulk copy stops at the array's end)
+          const int64_t G = args.K / kGroup;
+          const uint32_t inv_bytes =
+              args.inv_s == nullptr ? 0u
+                                    : static_cast<uint32_t>((G - g < L::kPG ? G - g : L::kPG) *
+                                                            kGroup * 4);
+          mbar_arrive_expect_tx(&pfull[ps],
+                                L::kPBytes + (args.sz_tma ? L::kSZBytes : 0) + inv_bytes);
           tma_load_2d(smem + L::kPOff + ps * L::kPBytes, &tmap_a, &pfull[ps],
                       g * (L::kPGroupBytes / 4), row0);
+          if (inv_bytes != 0 && AWQ_IN_BOUNDS(g < G && inv_bytes <= L::kInvBytes))
+            bulk_load_1d(smem + L::kIOff + ps * L::kInvBytes, args.inv_s + g * kGroup, inv_bytes,
+                         &pfull[ps]);
           if (args.sz_tma) {
             uint8_t* sz = smem + L::kSZOff + ps * L::kSZBytes;
             tma_load_2d(sz, &tmap_s, &pfull[ps], row0, g);
