@@ -408,6 +408,18 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
       tma_prefetch_desc(&tmap_w);
       tma_prefetch_desc(&tmap_s);
       tma_prefetch_desc(&tmap_z);
+      {   // X and inv_s first (the consumers stage X as soon as the dependency wait returns):
+          // an L2 prefetch is coherent with the preceding kernel's writes (L2 is where they
+          // land), so the staging loads after the wait hit L2
+        const int64_t xb = static_cast<int64_t>(M) * K * 2;
+        for (int64_t off = 0; off < xb; off += 65536)
+          prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(X) + off,
+                           static_cast<uint32_t>(xb - off < 65536 ? xb - off : 65536));
+        if (inv_s != nullptr)
+          for (int64_t off = 0; off < K * 4; off += 65536)
+            prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(inv_s) + off,
+                             static_cast<uint32_t>(K * 4 - off < 65536 ? K * 4 - off : 65536));
+      }
       int slot = 0, chunk = 0;
       uint32_t ph = 0;
       int64_t tile = t0;
@@ -438,16 +450,6 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
         const int64_t bytes = (r1 - r0) * row_bytes;
         for (int64_t off = 0; off < bytes; off += 65536)
           prefetch_l2_bulk(wrow + off, static_cast<uint32_t>(bytes - off < 65536 ? bytes - off : 65536));
-        // X and inv_s too: an L2 prefetch is coherent with the preceding kernel's writes
-        // (L2 is where they land), and the staging loads after the wait then hit L2
-        const int64_t xb = static_cast<int64_t>(M) * K * 2;
-        for (int64_t off = 0; off < xb; off += 65536)
-          prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(X) + off,
-                           static_cast<uint32_t>(xb - off < 65536 ? xb - off : 65536));
-        if (inv_s != nullptr)
-          for (int64_t off = 0; off < K * 4; off += 65536)
-            prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(inv_s) + off,
-                             static_cast<uint32_t>(K * 4 - off < 65536 ? K * 4 - off : 65536));
       }
       pdl_wait();
       AWQ_TRACE_AT(rec, kTrWaited, globaltimer_ns());
