@@ -83,14 +83,14 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, in
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, ASrc kA, Epi kEpi, bool kBf16 = false>
-awq_status launch_tc(const void* Xop, int64_t M, const void* Aop, int64_t a_rows,
-                     const awq::TcArgs& args, cudaStream_t st, const void* Aop2 = nullptr) {
-  using L = awq::TcLayout<BN, kA>;
+template <int BN, ASrc kA, Epi kEpi, bool kBf16, int kBlkT>
+awq_status launch_tc_blk(const void* Xop, int64_t M, const void* Aop, int64_t a_rows,
+                         const awq::TcArgs& args, cudaStream_t st, const void* Aop2) {
+  using L = awq::TcLayout<BN, kA, kBlkT>;
   static std::atomic<bool> attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AWQ_ERR_CUDA;
-  auto kern = awq::tc_gemm_kernel<BN, kA, kEpi, kBf16>;
+  auto kern = awq::tc_gemm_kernel<BN, kA, kEpi, kBf16, kBlkT>;
   if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem) !=
         cudaSuccess)
@@ -161,6 +161,23 @@ awq_status launch_tc(const void* Xop, int64_t M, const void* Aop, int64_t a_rows
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, tx, ta, ts, tz, a) != cudaSuccess) return AWQ_ERR_CUDA;
   return launch_status();
+}
+
+// Packed sources take stages of two 64-k blocks where the builders or the single MMA-issuing
+// thread set the pace: token tiles up to 128, and inv_s folded into the weights. Plain
+// BN = 256 keeps four one-block stages (two two-block stages, all that fit, measured slower
+// there: 1294 -> 1172 TFLOP/s on [28672, 8192] at M = 4096).
+template <int BN, ASrc kA, Epi kEpi, bool kBf16 = false>
+awq_status launch_tc(const void* Xop, int64_t M, const void* Aop, int64_t a_rows,
+                     const awq::TcArgs& args, cudaStream_t st, const void* Aop2 = nullptr) {
+  constexpr bool kPk = kA == ASrc::kPacked4 || kA == ASrc::kPacked3;
+  if constexpr (kPk && BN == 256) {
+    if (args.inv_s == nullptr)
+      return launch_tc_blk<BN, kA, kEpi, kBf16, 1>(Xop, M, Aop, a_rows, args, st, Aop2);
+    return launch_tc_blk<BN, kA, kEpi, kBf16, 2>(Xop, M, Aop, a_rows, args, st, Aop2);
+  } else {
+    return launch_tc_blk<BN, kA, kEpi, kBf16, kPk ? 2 : 1>(Xop, M, Aop, a_rows, args, st, Aop2);
+  }
 }
 
 template <ASrc kA, Epi kEpi, bool kBf16 = false>

@@ -9,9 +9,10 @@
 // side is BN tokens, so D = W_tile * X_tile^T lands in TMEM as 128 lanes (one per output
 // feature) x BN fp32 columns (one per token), and each dequantized weight is reused across
 // BN tokens. Persistent: one CTA per SM walks the (tile, K slice) work units in a grouped
-// order (see tile_of_block) with a shared-memory ring of 64-wide K stages that runs on
-// across tiles, and two TMEM accumulators so a tile's epilogue overlaps the next tile's
-// main loop:
+// order (see tile_of_block) with a shared-memory ring of K stages that runs on across tiles
+// (a stage is one 64-k block, or for packed sources two: a whole 128-k group, so the MMA
+// thread's per-stage waits and commit are paid once per eight MMAs), and two TMEM
+// accumulators so a tile's epilogue overlaps the next tile's main loop:
 //   warp 5       TMA producer: X slice (128-byte swizzle), and both parts of the A slice
 //                (two-part fp16 source);
 //   warp 1       TMEM allocator and single-thread tcgen05.mma issuer (kind::f16, fp32 acc);
@@ -71,21 +72,27 @@ enum class ASrc : int { kPacked4 = 0, kPacked3 = 1, kSplit16 = 2, kPair16 = 3, k
 // D[n][j] * e'[n][j], the recombined product times the row's own error operand.
 enum class Epi : int { kStoreY = 0, kRowSumSq = 1, kSiluMul = 2, kStoreF32 = 3, kGramDot = 4 };
 
-template <int BN, ASrc kA>
+template <int BN, ASrc kA, int kBlkT = 1>
 struct TcLayout {
   static constexpr bool kPk = kA == ASrc::kPacked4 || kA == ASrc::kPacked3;
   static constexpr int kXParts = kA == ASrc::kGram ? 2 : 1;   // B tiles per stage
   static constexpr int kAParts = (kPk || kA == ASrc::kFp16x1) ? 1 : 2;   // A tiles (and
                                                                        // accumulators) per stage
+  // packed sources with kBlkT = 2: two 64-k blocks (one 128-k group) per pipeline stage, so
+  // the single MMA-issuing thread waits and commits once per eight MMAs instead of four
+  static constexpr int kBlk = kPk ? kBlkT : 1;
   static constexpr int kXPartBytes = BN * kTcBK * 2;
-  static constexpr int kXBytes = kXParts * kXPartBytes;
+  static constexpr int kXBlockBytes = kXParts * kXPartBytes;
+  static constexpr int kXBytes = kBlk * kXBlockBytes;   // per stage
   static constexpr int kStages =
       kA == ASrc::kGram ? (BN >= 256 ? 2 : BN >= 128 ? 3 : 4)
       : kA == ASrc::kFp16x1 ? (BN >= 256 ? 4 : 6)
       : !kPk ? (BN >= 256 ? 3 : BN >= 128 ? 4 : BN >= 64 ? 5 : 6)
-             : (BN >= 256 ? 4 : BN >= 64 ? 5 : 6);
+             : kBlk == 2 ? (BN >= 128 ? 2 : 3)   // packed, stages of two blocks
+                         : (BN >= 256 ? 4 : BN >= 64 ? 5 : 6);
   static constexpr int kAPartBytes = kTcBM * kTcBK * 2;
-  static constexpr int kABytes = kAParts * kAPartBytes;
+  static constexpr int kABlockBytes = kAParts * kAPartBytes;
+  static constexpr int kABytes = kBlk * kABlockBytes;   // per stage
   // packed source: kPG groups (2 kPG stages) per ring slot
   static constexpr int kPG = !kPk ? 1 : BN <= 64 ? 4 : BN <= 128 ? 2 : 1;
   static constexpr int kPGroupBytes = kA == ASrc::kPacked4 ? 64 : kA == ASrc::kPacked3 ? 48 : 0;
@@ -254,13 +261,13 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
   return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
 
-template <int BN, ASrc kA, Epi kEpi, bool kBf16 = false>
+template <int BN, ASrc kA, Epi kEpi, bool kBf16 = false, int kBlkT = 1>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                    const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_s,
                    const __grid_constant__ CUtensorMap tmap_z, const TcArgs args) {
-  using L = TcLayout<BN, kA>;
+  using L = TcLayout<BN, kA, kBlkT>;
   constexpr int S = L::kStages;
   constexpr bool kPacked = L::kPk;
   extern __shared__ uint8_t smem_raw[];
@@ -346,15 +353,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const TcUnit t = unit_of(u, args);
         const int64_t m0 = static_cast<int64_t>(t.m_tile) * BN;
         const int64_t row0 = static_cast<int64_t>(t.row_tile) * kTcBM;
-        for (int i = 0; i < t.nkb; ++i) {
+        for (int i = 0; i < t.nkb; i += L::kBlk) {
           const int kb = t.kb0 + i;
           if (!mbar_wait(&empty[s], ph ^ 1)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full[s], L::kTxBytes);
-          tma_load_2d(smem + L::kXOff + s * L::kXBytes, &tmap_x, &full[s], kb * kTcBK,
-                      static_cast<int32_t>(m0));
+#pragma unroll
+          for (int b = 0; b < L::kBlk; ++b)
+            tma_load_2d(smem + L::kXOff + s * L::kXBytes + b * L::kXBlockBytes, &tmap_x,
+                        &full[s], (kb + b) * kTcBK, static_cast<int32_t>(m0));
           if (kA == ASrc::kGram)   // the lo part of the normalised Gram matrix
             tma_load_2d(smem + L::kXOff + s * L::kXBytes + L::kXPartBytes, &tmap_x, &full[s],
                         static_cast<int32_t>(args.K) + kb * kTcBK, static_cast<int32_t>(m0));
@@ -391,16 +400,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!mbar_wait(&acc_empty[buf], acc_ph ^ 1)) break;   // epilogue released the buffer
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * L::kAParts * BN);
-        for (int i = 0; i < t.nkb; ++i) {
+        for (int i = 0; i < t.nkb; i += L::kBlk) {
           ok = mbar_wait(&full[s], ph);
           if (ok && kPacked) ok = mbar_wait(&built[s], ph);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + L::kAOff + s * L::kABytes);
-          const uint32_t x_base = smem_u32(smem + L::kXOff + s * L::kXBytes);
+#pragma unroll
+          for (int b = 0; b < L::kBlk; ++b) {
+          const uint32_t a_base = smem_u32(smem + L::kAOff + s * L::kABytes + b * L::kABlockBytes);
+          const uint32_t x_base = smem_u32(smem + L::kXOff + s * L::kXBytes + b * L::kXBlockBytes);
 #pragma unroll
           for (int kk = 0; kk < kTcBK / 16; ++kk) {
-            const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
+            const uint32_t acc = (i | b | kk) != 0 ? 1u : 0u;
             if (kA == ASrc::kGram) {
               // A_hi B_hi -> D_0; A_hi B_lo + A_lo B_hi -> D_1
               const uint64_t ah = sw128_kmajor_desc(a_base + kk * 32);
@@ -417,6 +428,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                            sw128_kmajor_desc(a_base + part * L::kAPartBytes + kk * 32),
                            sw128_kmajor_desc(x_base + kk * 32), idesc, acc);
             }
+          }
           }
           tc_commit(&empty[s]);
           if (++s == S) { s = 0; ph ^= 1; }
@@ -437,8 +449,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const TcUnit tu = unit_of(u, args);
         const int64_t n = static_cast<int64_t>(tu.row_tile) * kTcBM + r;
-        // one 128-k group per iteration: both of its 64-k stages are built, then one proxy
-        // fence and one arrival per stage (K slices are whole groups, so nkb is even)
+        // one 128-k group per iteration: the stage's two 64-k blocks are built, then one proxy
+        // fence and one arrival (K slices are whole groups, so nkb is even)
         for (int i = 0; i < tu.nkb; i += 2) {
           const int kb = tu.kb0 + i;
           uint32_t z = 0;
@@ -450,11 +462,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               sv = args.scales[g * N + n];
             }
           }
-          const int s1 = s + 1 == S ? 0 : s + 1;
-          const uint32_t ph1 = s + 1 == S ? (ph ^ 1u) : ph;
-          // the A slots are free once the MMAs that read them have completed; the X tiles of
-          // the stages are not needed here, so building overlaps their loads
-          bool got = mbar_wait(&empty[s], ph ^ 1) && mbar_wait(&empty[s1], ph1 ^ 1);
+          // the group's two 64-k blocks: one stage (kBlk = 2) or the two stages s and s1. A
+          // stage is free once the MMAs that read it have completed; its X blocks are not
+          // needed here, so building overlaps their loads
+          const int s1 = L::kBlk == 2 ? s : (s + 1 == S ? 0 : s + 1);
+          const uint32_t ph1 = L::kBlk == 2 ? ph : (s + 1 == S ? (ph ^ 1u) : ph);
+          bool got = mbar_wait(&empty[s], ph ^ 1);
+          if (L::kBlk == 1) got = got && mbar_wait(&empty[s1], ph1 ^ 1);
           if (got) got = mbar_wait(&pfull[ps], pph);
           ok = __all_sync(0xffffffffu, got);   // keep the warp converged for .aligned ops
           if (!ok) break;
@@ -483,7 +497,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         gi * kGroup;
 #pragma unroll
           for (int e = 0; e < 2; ++e) {             // stage i + e of the group
-            uint8_t* atile = smem + L::kAOff + (e ? s1 : s) * L::kABytes;
+            // block e: the second half of stage s (kBlk = 2), or stage s1
+            uint8_t* atile = L::kBlk == 2 ? smem + L::kAOff + s * L::kABytes + e * L::kABlockBytes
+                                          : smem + L::kAOff + (e ? s1 : s) * L::kABytes;
             if (kA == ASrc::kPacked4) {
               // row r of group gi: 64 bytes, this stage's 32 k at byte 32 * e + 16 * h
               const uint4 pw = *reinterpret_cast<const uint4*>(prow + gi * 64 + 32 * e + 16 * h);
@@ -521,7 +537,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           fence_proxy_async_smem();
           mbar_arrive(&built[s]);
-          mbar_arrive(&built[s1]);
+          if (L::kBlk == 1) mbar_arrive(&built[s1]);
           s = s1 + 1 == S ? 0 : s1 + 1;
           ph = s1 + 1 == S ? (ph1 ^ 1u) : ph1;
         }
