@@ -475,6 +475,24 @@ def profile_rows(awq, dev):
     torch.cuda.synchronize()
 
 
+def segment_launches(records):
+    """Splits the trace build's per-CTA records (in CTA start order) into launches. A
+    launch's CTAs all start before the next launch's first CTA (which launches only after
+    every CTA of this one has passed its dependency wait), and each blockIdx (word 6)
+    appears once per launch, so a launch ends where a blockIdx repeats."""
+    launches, cur, seen = [], [], set()
+    for rec in records:
+        b = int(rec[6])
+        if b in seen:
+            launches.append(np.array(cur))
+            cur, seen = [], set()
+        cur.append(rec)
+        seen.add(b)
+    if cur:
+        launches.append(np.array(cur))
+    return launches
+
+
 def trace_decode(awq, dev, l2, stream, steps):
     """The headline step (M = 1 on the three decode shapes, weights-ready, one CUDA graph) on
     the trace build: the per-launch timeline of the streaming decode kernel from its CTAs'
@@ -508,19 +526,7 @@ def trace_decode(awq, dev, l2, stream, steps):
         e1.record(stream)
     torch.cuda.synchronize()
     step_us = e0.elapsed_time(e1) * 1e3 / steps
-    R = awq.trace_read().astype(np.int64)
-    # a launch's CTAs all start before the next launch's first CTA (which launches only after
-    # every CTA of this one has passed its dependency wait); each blockIdx appears once
-    launches, cur, seen = [], [], set()
-    for rec in R:
-        b = int(rec[6])
-        if b in seen:
-            launches.append(np.array(cur))
-            cur, seen = [], set()
-        cur.append(rec)
-        seen.add(b)
-    if cur:
-        launches.append(np.array(cur))
+    launches = segment_launches(awq.trace_read().astype(np.int64))
     per = {j: [] for j in range(len(shapes))}
     for li in range(len(shapes), len(launches)):
         L, prev = launches[li], launches[li - 1]
