@@ -310,10 +310,12 @@ int tc_bn_for(int64_t M) { return M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 :
 // Split-K for the tensor-core GEMM when the output has too few 128 x BN tiles to occupy the
 // GPU (batched decode, small prefill). The persistent kernel runs one CTA per SM and hands
 // out (tile, K slice) units round-robin, so the busiest SM does ceil(tiles * s / sms) units
-// of K / s each: pick the split s that minimises that, i.e. ceil(tiles * s / sms) / s (a
-// later s must win by more than 2% per extra slice, since each slice adds 8 bytes of fp32
-// partial sums per output), with at least two 128-wide groups per slice and the partial
-// traffic within about the packed weight bytes.
+// of K / s each: pick the split s that minimises that, i.e. ceil(tiles * s / sms) / s, with
+// at least two 128-wide groups per slice and the partial traffic within about the packed
+// weight bytes. A later s must win by more than 12% per extra slice: each slice adds a
+// pipeline fill, an epilogue and 8 bytes of fp32 partial sums per output to reduce. On the
+// batched shapes 12% measured best among 2, 6, 12, 40 and 60% (e.g. [14336, 4096] at M = 32
+// runs unsplit, 26.6 -> 24.3 us; [4096, 14336] takes 4 slices instead of 9).
 int splitk_for(int64_t M, int64_t N, int64_t K) {
   const int64_t bn = tc_bn_for(M);
   const int64_t tiles = ((N + awq::kTcBM - 1) / awq::kTcBM) * ((M + bn - 1) / bn);
@@ -328,7 +330,7 @@ int splitk_for(int64_t M, int64_t N, int64_t K) {
   for (int64_t s = 2; s <= s_max; ++s) {
     const double cost =
         static_cast<double>((tiles * s + sms - 1) / sms) / static_cast<double>(s);
-    if (cost * (1.0 + 0.02 * static_cast<double>(s - best)) < best_cost) {
+    if (cost * (1.0 + 0.12 * static_cast<double>(s - best)) < best_cost) {
       best = static_cast<int>(s);
       best_cost = cost;
     }
