@@ -265,7 +265,7 @@ awq_status launch_gemv_stream_t(const void* x, int64_t M, const uint32_t* qweigh
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, tw, ts, tz, qweight, static_cast<const A*>(x),
+  if (cudaLaunchKernelEx(&cfg, kern, tw, ts, tz, static_cast<const A*>(x),
                          static_cast<int>(M), N, K, inv_s, static_cast<A*>(y), lay,
                          flags) != cudaSuccess)
     return AWQ_ERR_CUDA;

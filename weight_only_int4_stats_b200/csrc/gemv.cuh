@@ -207,9 +207,12 @@ namespace awq {
 // Streaming decode GEMM (the decode path for M <= 16; N in whole 16-row tiles and X within
 // one CTA's shared memory).
 //
-// Persistent: the grid is one CTA per SM (as many as there are 16-row tiles, at most) and
-// CTA b owns the contiguous range of whole 16-row tiles [b*T/P, (b+1)*T/P), so no output is
-// split across CTAs and the result does not depend on the grid. One producer thread walks
+// Persistent: the grid is one or two CTAs per SM (as many as there are 16-row tiles, at
+// most). Each CTA owns a contiguous range of whole 16-row tiles, floor(T/P) of them plus one
+// for the first T mod P CTAs, so no output is split across CTAs and the result does not
+// depend on the grid. (With boundaries at b*T/P instead, CTAs b and b + P/2, which a grid of
+// two per SM usually places on one SM, got equal counts: at 688 tiles over 296 CTAs, 48 SMs
+// ran six tiles while the rest ran four.) One producer thread walks
 // the CTA's (tile, 2048-k chunk) units and streams each unit's packed weights (16 rows x
 // 1 KB at 4 bits, 768 B at 3 bits), fp16 scales and uint8 zeros ([16 groups, 16 rows]) with
 // TMA into a shared-memory ring. The packed weights arrive as 128-byte-wide boxes with the
@@ -224,11 +227,12 @@ namespace awq {
 // Back-to-back launches overlap (programmatic dependent launch). A CTA needs at most half of
 // an SM's shared memory, so the next GEMM's CTAs become resident beside this one's as soon as
 // every CTA of this grid has passed griddepcontrol.wait (where the next launch is allowed).
-// Before the wait a CTA touches no output and no activation: it issues L2 prefetches of its
-// weight rows, of X and of inv_s (coherent with writes of the preceding kernel, so always
-// safe) and, when the
+// Before the wait a CTA touches no output and no activation: it issues L2 prefetches of X
+// and of inv_s (coherent with writes of the preceding kernel, so always safe) and, when the
 // caller states that the weights are not written by the kernel launched just before
-// (kGemvWeightsReady), TMA-loads the first ring slots.
+// (kGemvWeightsReady), TMA-loads the first ring slots. An L2 prefetch of the CTA's weight
+// rows as well measured slower, with or without the early ring loads: it competes with them
+// and with the preceding kernel's stream.
 //
 // After the wait the consumer warps stage X ([M, K], small at decode; each thread issues all
 // its loads of a round at once) from global memory into shared memory in the order the MMA's
@@ -344,7 +348,7 @@ __device__ __forceinline__ void dequant_word_qz_bf16(uint32_t w, uint32_t bias, 
 template <int kNTiles, bool kOffset, bool kBf16 = false, int kBits = 4>
 __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
-    const __grid_constant__ CUtensorMap tmap_z, const uint32_t* __restrict__ qweight,
+    const __grid_constant__ CUtensorMap tmap_z,
     const act_t<kBf16>* __restrict__ X, int M, int64_t N, int64_t K,
     const float* __restrict__ inv_s, act_t<kBf16>* __restrict__ Y, G4Smem lay, unsigned flags) {
   static_assert(kBits == 4 || kBits == 3, "4- or 3-bit codes");
@@ -371,7 +375,8 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
   const int lane = threadIdx.x & 31;
   const int64_t T = (N + kGemvRows - 1) / kGemvRows;
   const int64_t P = gridDim.x;
-  const int64_t t0 = blockIdx.x * T / P, t1 = (blockIdx.x + 1) * T / P;
+  const int64_t bx = blockIdx.x, tq = T / P, tr = T % P;
+  const int64_t t0 = bx * tq + (bx < tr ? bx : tr), t1 = t0 + tq + (bx < tr ? 1 : 0);
   const int Ki = static_cast<int>(K);
   const int G = Ki / kGroup;
   const int C = (Ki + kG4KC - 1) / kG4KC;
@@ -442,14 +447,6 @@ __global__ void __launch_bounds__(kG4Threads, 2) gemv_stream_kernel(
         // the weights do not depend on the preceding kernel: fill the (empty) ring now
         const int64_t n_early = units < S ? units : S;
         for (; u < n_early; ++u) issue();
-      }
-      {   // HBM -> L2 for this CTA's weight rows (one contiguous range)
-        const int64_t row_bytes = K * kBits / 8;
-        const int64_t r0 = t0 * kGemvRows, r1 = t1 * kGemvRows < N ? t1 * kGemvRows : N;
-        const uint8_t* wrow = reinterpret_cast<const uint8_t*>(qweight) + r0 * row_bytes;
-        const int64_t bytes = (r1 - r0) * row_bytes;
-        for (int64_t off = 0; off < bytes; off += 65536)
-          prefetch_l2_bulk(wrow + off, static_cast<uint32_t>(bytes - off < 65536 ? bytes - off : 65536));
       }
       pdl_wait();
       AWQ_TRACE_AT(rec, kTrWaited, globaltimer_ns());
