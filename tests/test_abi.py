@@ -115,6 +115,22 @@ def test_gemm_workspace_follows_the_chosen_kernel():
         assert ws >= 2 * M * N * 4 and ws % 256 == 0, (M, N, K, ws)
 
 
+@pytest.mark.parametrize("N,K,M,slices", [
+    (14336, 4096, 32, 1), (14336, 4096, 64, 1), (14336, 4096, 128, 1), (14336, 4096, 256, 1),
+    (4096, 14336, 32, 4), (4096, 14336, 64, 4), (4096, 14336, 128, 4), (4096, 14336, 256, 4),
+    (6144, 4096, 32, 3), (6144, 4096, 64, 3), (6144, 4096, 128, 3), (6144, 4096, 256, 2),
+])
+def test_split_k_choice_on_the_batched_shapes(N, K, M, slices):
+    # the split-K chooser on 148 SMs (the count the library assumes without a device, and a
+    # B200's): a larger split has to win by 12 % per extra slice. On B200 this beat 2, 6, 40
+    # and 60 %: [14336, 4096] at M = 32 / 64 runs unsplit (26.6 -> 24.3, 29.4 -> 26.2 us
+    # against 5 slices), [4096, 14336] takes 4 slices, not 9 (2 or 3 were 20-60 % slower).
+    # The workspace holds one fp32 partial M x N per slice when K is split, nothing otherwise.
+    ws = _lib().awq_gemm_workspace_size(M, N, K, 4)
+    want = 0 if slices == 1 else -(-slices * M * N * 4 // 256) * 256
+    assert ws == want, (N, K, M, ws, want)
+
+
 def test_gemm_workspace_is_checked_before_launch():
     # the tensor-core path with few output tiles needs room for split-K partial sums; a
     # missing or short workspace is rejected on the host (AWQ_ERR_WORKSPACE) before anything
