@@ -165,6 +165,16 @@ def test_gemm_decode(awq, M, N, K):
     _check_gemm(awq, X, qw, sc, z, N, K)
 
 
+@pytest.mark.parametrize("N,K", [(4800, 8320), (64, 16512), (48, 8192)])
+def test_gemm_decode_m1_long_k(awq, N, K):
+    # M = 1 with X longer than one staging round (8192 values): a ragged last round (8320),
+    # two further rounds (16512) and exactly one round (8192); 300 tiles of 16 rows is more
+    # than the grid holds, so some CTAs own two tiles
+    W, X, m = rand_layer(N + K, N, K, 1, outliers=False)
+    qw, sc, z = _packed(W, np.sqrt(m).astype(np.float32))
+    _check_gemm(awq, X, qw, sc, z, N, K)
+
+
 @pytest.mark.parametrize("M", [1, 16])
 def test_gemm_decode_inv_s(awq, M):
     N, K = 96, 512
